@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark of the sm_100a Mamba-2 SSD hot path (prefill + cached decode).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (per rank; ranks process independent batches, so scaling is weak):
+  * prefill, the headline: the 2.7B-layer shape -- b=8 sequences x T=4096 tokens,
+    H=80 heads, P=64, N=128, G=1, chunk 256, bf16 x/B/C, fp32 dt/A/D, h0 ~ N(0, 0.1).
+    One step = one ssd_prefill call over that batch.  value = algorithmic TFLOP/s.
+  * cached decode at the 2.7B shape: 64 layers x (80 x 64 x 128) fp32 state + width-4
+    conv over 5376 channels, batch 1 (and 32), state from the prefill's final state,
+    run as graph launches of on-device steps; reported under "decode".
+Inputs are seeded synthetic draws (ssd_inputs); the per-step prefill inputs (740 MB)
+exceed the 126 MB L2, so no flush is needed between steps.
+
+Prints ONE JSON line on rank 0.  --impl reference times the CPU oracle (the only
+reference this method has: an fp64 C implementation of the recurrence) on bounded
+samples of the same workload, in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSD prefill TFLOP/s + tokens/s; decode steps/s + HBM GB/s; % of roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# prefill workload (the 2.7B-layer configuration)
+PB, PT, PH, PP, PN, PG, PL = 8, 4096, 80, 64, 128, 1, 256
+# decode workload (the 2.7B-shaped cache)
+DL, DH, DP, DN, DG, DK = 64, 80, 64, 128, 1, 4
+
+
+def peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ----------------------------------------------------------------------------- work counts
+def prefill_flops(b, T, H, P, N, G, L):
+    """Algorithmic FLOPs of the chunked dual form: per chunk and group the causal C.B^T
+    triangle (diagonal included); per chunk and head the masked product with X (same
+    triangle), the chunk state and the state-to-output term; plus the O(P N) scan."""
+    nc_full, rem = divmod(T, L)
+    lens = [L] * nc_full + ([rem] if rem else [])
+    tri = sum(l * (l + 1) // 2 for l in lens)
+    f = 2.0 * b * G * tri * N            # C.B^T, causal triangle, once per group
+    f += 2.0 * b * H * tri * P           # (C.B^T o L) X
+    f += 2.0 * b * H * T * P * N         # chunk states
+    f += 2.0 * b * H * T * N * P         # state-to-output
+    f += 2.0 * b * H * len(lens) * P * N  # inter-chunk recurrence
+    return f
+
+
+def prefill_bytes(b, T, H, P, N, G, io_bytes=2, with_h0=True):
+    """Algorithmic HBM bytes: x, B, C, dt in, y out, h0 in, h_final out."""
+    tok = b * T
+    by = tok * H * P * io_bytes * 2 + tok * G * N * io_bytes * 2 + tok * H * 4
+    by += b * H * P * N * 4 * (2 if with_h0 else 1) + 2 * H * 4
+    return float(by)
+
+
+def decode_bytes_per_step(layers, b, H, P, N, G, k=4, io_bytes=2):
+    """State read+write, conv state read+write, step inputs, conv weights, A/D, y."""
+    Dc = H * P + 2 * G * N
+    st = 2.0 * layers * b * H * P * N * 4
+    cv = 2.0 * layers * b * Dc * (k - 1) * 4
+    inp = layers * b * (Dc * io_bytes + H * 4)
+    w = layers * (Dc * k * 4 + Dc * 4 + 2 * H * 4)
+    y = layers * b * H * P * io_bytes
+    return st + cv + inp + w + y
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+        self.windows = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if self.windows and not any(a - 0.15 <= ts <= b + 0.15 for a, b in self.windows):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def sha_prefix(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:12]
+
+
+def dram_traffic(kernel):
+    """Per-launch DRAM bytes of `kernel` from profiles/dram_traffic.txt, only if the source
+    file recorded there is unchanged since the ncu capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        parts = line.split()
+        if len(parts) >= 4 and parts[0] == kernel:
+            src, sha, per_launch = parts[1], parts[2], float(parts[3])
+            full = os.path.join(ROOT, src)
+            if os.path.exists(full) and sha_prefix(full) == sha:
+                return per_launch
+    return None
+
+
+def oracle_prefill_sample(case, heads, seqs=(0,)):
+    """Time the fp64 oracle recurrence on a (sequence x head) subset; returns seconds."""
+    import oracle
+    hpg = case.H // case.G
+    x = case.x[list(seqs)][:, :, heads]
+    dt = case.dt[list(seqs)][:, :, heads]
+    B = case.B[list(seqs)][:, :, [h // hpg for h in heads]]
+    C = case.C[list(seqs)][:, :, [h // hpg for h in heads]]
+    h0 = None if case.h0 is None else case.h0[list(seqs)][:, heads]
+    oracle.ssd_recurrence(x[:, :64], dt[:, :64], case.A[heads], B[:, :64], C[:, :64], case.D[heads], h0)
+    t0 = time.perf_counter()
+    oracle.ssd_recurrence(x, dt, case.A[heads], B, C, case.D[heads], h0)
+    return time.perf_counter() - t0, oracle.max_threads()
+
+
+def cpu_baseline(case, flops_per_tokhead, target_s=10.0):
+    """The oracle as it stands on the host cores, on a bounded sample of the workload:
+    8 heads of sequence 0 first, then as many (sequence, head) pairs as fit ~target_s."""
+    t8, cores = oracle_prefill_sample(case, list(range(8)))
+    pairs = int(min(case.b * case.H, max(8, 8 * target_s / max(t8, 1e-3))))
+    seqs = max(1, min(case.b, pairs // case.H))
+    heads = list(range(min(case.H, pairs if seqs == 1 else case.H)))
+    t, cores = oracle_prefill_sample(case, heads, tuple(range(seqs)))
+    n = seqs * len(heads)
+    return {"value": flops_per_tokhead * case.T * n / t / 1e12, "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle", "seconds": t,
+            "sample": "fp64 oracle recurrence on %d sequence(s) x %d heads x %d tokens of this workload (%.1f s), "
+                      "scaled by the algorithmic FLOPs per token-head" % (seqs, len(heads), case.T, t)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from ssd_inputs import make_config
+    case = make_config("mamba2_2p7b_layer")
+    flops_per_tokhead = prefill_flops(PB, PT, PH, PP, PN, PG, PL) / (PB * PT * PH)
+    heads = list(range(8))
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt_s, cores = oracle_prefill_sample(case, heads)
+        if i >= args.warmup:
+            times.append(dt_s)
+    t = statistics.median(times)
+    tokheads = PT * len(heads)
+    value = flops_per_tokhead * tokheads / t / 1e12
+    sample = "fp64 oracle recurrence, sequence 0 x heads 0-7 x 4096 tokens of the 2.7B-layer prefill per step"
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "mamba2_2p7b_layer_prefill", "b": PB, "T": PT, "H": PH, "P": PP, "N": PN,
+                       "G": PG, "chunk": PL},
+            "tokens_per_s": tokheads / PH / t,
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=1024, help="timed decode steps at batch 1")
+    ap.add_argument("--decode-batches", default="1,32")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    import state_space_model_04_b200 as ssd
+    from ssd_inputs import make_config
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    pk, pk_kind = peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---------------- prefill inputs (seeded per rank: independent batches)
+    case = make_config("mamba2_2p7b_layer", seed=2 + 1000 * rank)
+    def bf(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    host = {"x": bf(case.x_bits), "B": bf(case.B_bits), "C": bf(case.C_bits),
+            "dt": torch.from_numpy(case.dt), "A": torch.from_numpy(case.A), "D": torch.from_numpy(case.D),
+            "h0": torch.from_numpy(case.h0)}
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    d = {k: v.to(dev) for k, v in host.items()}
+    y = torch.empty_like(d["x"])
+    hf = torch.empty_like(d["h0"])
+    ws = torch.empty(ssd.prefill_workspace_size(PB, PT, PH, PP, PN, PG, PL, ssd.SSD_BF16), dtype=torch.uint8, device=dev)
+
+    def prefill_step():
+        ssd.prefill(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], chunk=PL, h0=d["h0"], y=y, h_final=hf,
+                    workspace=ws)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(args.warmup):
+        prefill_step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    n0 = ssd.launch_count()
+    ssd.profile_begin()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        prefill_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(w0, time.time())
+    kt = ssd.profile_end()
+    launches = ssd.launch_count() - n0
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    flops = prefill_flops(PB, PT, PH, PP, PN, PG, PL)
+    pbytes = prefill_bytes(PB, PT, PH, PP, PN, PG)
+    tflops = flops * world / (ms * 1e-3) / 1e12
+    tokens_s = PB * PT * world / (ms * 1e-3)
+
+    # dominant kernel: the one with the largest summed event time in the timed region
+    dom = max(kt.items(), key=lambda kv: kv[1][1])
+    dom_name, (dom_n, dom_ms) = dom
+    dom_avg_ms = dom_ms / max(dom_n, 1)
+    per_kernel_bytes = {
+        # fused or not, the algorithmic bytes of one launch of the dominant prefill kernel
+        "ssd_prefill_fused": pbytes,
+        "simt_chunk_output": pbytes - PB * PH * PP * PN * 4 + PB * ((PT + PL - 1) // PL) * PH * PP * PN * 4,
+    }
+    alg = per_kernel_bytes.get(dom_name, pbytes)
+    achieved = alg / (dom_avg_ms * 1e-3) / 1e9
+    hbm_peak = pk["hbm_gbs"]
+    roofline = {"kernel": dom_name, "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": dram_traffic(dom_name),
+                "peak_source": pk_kind + " (hbm_gbs, burst copy)", "avg_launch_ms": dom_avg_ms,
+                "tensor_tflops": flops / (dom_avg_ms * 1e-3) / 1e12 if dom_name == "ssd_prefill_fused" else None,
+                "tensor_frac_of_bf16_peak": (flops / (dom_avg_ms * 1e-3) / 1e12 / pk["bf16_tflops"])
+                if dom_name == "ssd_prefill_fused" else None,
+                "kernels": {k: {"launches": v[0], "avg_ms": v[1] / max(v[0], 1)} for k, v in kt.items()}}
+
+    # ---------------- e2e through the public API with host buffers
+    out_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    out_h = torch.empty(hf.shape, dtype=hf.dtype).pin_memory()
+
+    def e2e_step():
+        for k in d:
+            d[k].copy_(pinned[k], non_blocking=True)
+        prefill_step()
+        out_y.copy_(y, non_blocking=True)
+        out_h.copy_(hf, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    w0 = time.time()
+    e2[0].record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e2[1].record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(w0, time.time())
+    barrier()
+    ms_e2e = max_over_ranks(e2[0].elapsed_time(e2[1]) / args.steps)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = y.numel() * y.element_size() + hf.numel() * hf.element_size()
+    e2e = {"value": flops * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+
+    # ---------------- cached decode (state from this prefill's final state)
+    decode = {}
+    for db in [int(v) for v in args.decode_batches.split(",") if v]:
+        box = [0]
+        decode["b%d" % db] = bench_decode(ssd, torch, dev, stream, case, hf, db, args, clocks, barrier,
+                                          max_over_ranks, world, pk, box)
+        launches += box[0]
+
+    clk = clocks.stop()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(case, flops / (PB * PT * PH))
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "mamba2_2p7b_layer_prefill", "b": PB, "T": PT, "H": PH, "P": PP, "N": PN,
+                           "G": PG, "chunk": PL, "global_batch": PB * world, "seq_len": PT,
+                           "parallelism": "dp%d" % world,
+                           "l2": "inputs larger than L2 (%.0f MB per step vs 126 MB)" % (pbytes / 1e6)},
+                "tokens_per_s": tokens_s, "flops_per_step": flops, "bytes_per_step": pbytes,
+                "hbm_gbs_alg": pbytes * world / (ms * 1e-3) / 1e9,
+                "tensor_frac": tflops / world / pk["bf16_tflops"],
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+                "clocks": clk, "decode": decode}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_decode(ssd, torch, dev, stream, case, hf, b, args, clocks, barrier, max_over_ranks, world, pk, box):
+    from ssd_inputs import make_decode_params
+    Dc = DH * DP + 2 * DG * DN
+    A, D, conv_w, conv_b, dt_bias = make_decode_params(DL, DH, DP, DN, DG, DK, seed=3)
+    A, D, conv_w, conv_b = (torch.from_numpy(v).to(dev) for v in (A, D, conv_w, conv_b))
+    # state: the prefill's final state of sequence r mod 8, every layer
+    h = hf[torch.arange(b, device=dev) % hf.shape[0]].unsqueeze(0).expand(DL, b, DH, DP, DN).contiguous()
+    # conv window: the last k-1 tokens of that sequence's [x | B | C]
+    rows = []
+    for r in range(b):
+        s = r % case.b
+        xs = case.x[s, -3:].reshape(3, -1)
+        bs = case.B[s, -3:].reshape(3, -1)
+        cs_ = case.C[s, -3:].reshape(3, -1)
+        rows.append(np.concatenate([xs, bs, cs_], 1).T)
+    cst = torch.from_numpy(np.stack(rows)).to(dev).unsqueeze(0).expand(DL, b, Dc, 3).contiguous()
+    ring = 256 if b == 1 else 32
+    from ssd_inputs import make_decode_ring_device
+    xbc, dt = make_decode_ring_device(ring, DL, b, DH, DP, DN, DG, dt_bias, seed=77, device=dev)
+    steps_per_launch = min(args.decode_steps if b == 1 else 64, 512)
+    plan = ssd.DecodePlan(h, cst, xbc, dt, A, D, conv_w, conv_b, n_steps=steps_per_launch, G=DG)
+    plan.launch()
+    torch.cuda.synchronize()
+    launches_timed = max(1, (args.decode_steps if b == 1 else 128) // steps_per_launch)
+    barrier()
+    n0 = ssd.launch_count()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    w0 = time.time()
+    ev[0].record(stream)
+    for _ in range(launches_timed):
+        plan.launch()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    clocks.mark(w0, time.time())
+    box[0] = ssd.launch_count() - n0
+    barrier()
+    ms = max_over_ranks(ev[0].elapsed_time(ev[1]))
+    steps = launches_timed * steps_per_launch
+    sps = steps * world / (ms * 1e-3)
+    byt = decode_bytes_per_step(DL, b, DH, DP, DN, DG)
+    gbs = byt * sps / 1e9
+    ok = bool(torch.isfinite(h).all().item())
+    plan.close()
+    del h, cst, xbc, dt
+    torch.cuda.empty_cache()
+    return {"batch": b, "layers": DL, "steps": steps, "steps_per_launch": steps_per_launch,
+            "steps_per_s": sps, "tokens_per_s": sps * b, "ms_per_step": ms / steps,
+            "bytes_per_step": byt, "hbm_gbs_alg": gbs, "hbm_frac": gbs / world / pk["hbm_gbs"],
+            "kernel": "decode_step (graph of %d steps)" % steps_per_launch, "state_finite": ok}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,188 @@
+/*
+ * ssd.h -- C ABI of libssd_b200.so, the sm_100a (B200) Mamba-2 SSD hot path.
+ *
+ * Method: "Compiler-First State Space Duality and Portable O(1) Autoregressive Caching"
+ * (arXiv 2603.09555), cited below as [CF-SSD].
+ *   - ssd_prefill: the chunked SSD prefill -- per-head scalar decay a = dt*A, its
+ *     segment-wise prefix sum exponentiated into the lower-triangular decay matrix, the
+ *     intra-chunk dual form (Eq. 3), chunk summary states, the sequential inter-chunk
+ *     recurrence, the state-to-output term and the D skip ("Chunked recurrence" and
+ *     "Diagonal state matrix" properties).  Its final state initialises the decode cache
+ *     (O(1) caching section).
+ *   - ssd_decode_step / decode plans: the O(1) cached decode step -- a width-k causal
+ *     depthwise conv over k-1 cached inputs, then one recurrence step
+ *     h <- exp(dt*A) h + dt * x B^T, y = h C + D x (O(1) caching section), looped on the
+ *     device with no host round trip per token ("Compiled on-device loops").
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library never
+ *     frees or retains them past the call (a decode plan retains the pointers it was
+ *     created with until it is destroyed).  Layouts are row-major (last index
+ *     contiguous), densely packed, and every pointer must be 16-byte aligned.
+ *   - Scalars per head (dt, A, D), states (h0, h_final, h, conv_state) and conv
+ *     parameters are fp32.  x, B, C, y (prefill) and xbc, y (decode) use the io dtype
+ *     (SSD_BF16: bfloat16 payloads; SSD_F32: float).
+ *   - The library allocates no device memory per call: scratch comes from the caller's
+ *     workspace, sized by the matching *_workspace_size query.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; the call returns once it is enqueued.
+ *   - Every entry point validates its arguments on the host before launching anything
+ *     and returns a status; nothing aborts and nothing throws across the ABI.
+ *     ssd_last_error() returns a human-readable detail for the calling thread's last
+ *     failure.  Asynchronous CUDA failures surface as SSD_ERR_CUDA on a later call.
+ *   - Prefill requires P == 64 and N in {64, 128}; decode requires P == 64 and
+ *     N in {64, 128}; any other shape returns SSD_ERR_UNSUPPORTED.
+ */
+#ifndef SSD_B200_H_
+#define SSD_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,  /* null pointer, bad dimension, misalignment, bad enum */
+    SSD_ERR_UNSUPPORTED = 2,  /* valid but not implemented shape (e.g. P != 64)     */
+    SSD_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                  */
+    SSD_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up                 */
+    SSD_ERR_WORKSPACE = 5,    /* workspace pointer null or smaller than required    */
+    SSD_ERR_INTERNAL = 6      /* a device-side consistency check failed             */
+} ssd_status;
+
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+typedef enum { SSD_ACT_NONE = 0, SSD_ACT_SILU = 1 } ssd_act;
+
+/* Library version as 10000*major + 100*minor + patch. */
+SSD_API int ssd_version(void);
+
+/* Static description of a status code (never NULL). */
+SSD_API const char* ssd_status_string(int status);
+
+/* Detail of the calling thread's most recent non-OK status ("" if none). */
+SSD_API const char* ssd_last_error(void);
+
+/* ------------------------------------------------------------------------------------
+ * Prefill  ([CF-SSD] Eq. 3, "Chunked recurrence", O(1) caching: prefill fills the cache)
+ *
+ * Shapes: b sequences of T tokens, H heads of head dim P, state size N, G groups of
+ * B/C (head h reads group h / (H/G)), chunk length `chunk`.
+ *   x       [b][T][H][P]  io dtype      dt [b][T][H] fp32 (positive step sizes, i.e.
+ *                                        already passed through softplus)
+ *   A       [H] fp32 (negative)         D  [H] fp32
+ *   B, C    [b][T][G][N]  io dtype
+ *   h0      [b][H][P][N]  fp32, or NULL for a zero initial state
+ *   y       [b][T][H][P]  io dtype      (output)
+ *   h_final [b][H][P][N]  fp32, or NULL to skip (output; may alias h0 exactly)
+ * Computes, per (sequence, head), the result of the recurrence
+ *   h_t = exp(dt_t A) h_{t-1} + dt_t x_t B_t^T,  y_t = h_t C_t + D x_t,  h_{-1} = h0
+ * through the chunked dual form.  T need not be a multiple of `chunk`: the last chunk
+ * is then shorter.  T == 0 or b == 0 is a no-op apart from h_final = h0 (or zeros).
+ * chunk must be 64, 128 or 256.  x, B, C, dt, A, D must not alias y or h_final.
+ * Arithmetic: SSD_BF16 inputs use bf16 tensor-core contractions (tcgen05) with fp32
+ * accumulation, fp32 decay in log space and an fp32 running state; SSD_F32 inputs use
+ * fp32 FMA with the prefix sums of dt*A kept in fp64 (no TF32 anywhere).
+ * Errors: SSD_ERR_INVALID_ARG (null pointer for a required argument, negative size,
+ * H % G != 0, bad chunk or dtype, misaligned pointer), SSD_ERR_UNSUPPORTED (P, N),
+ * SSD_ERR_WORKSPACE (workspace too small or NULL while required), SSD_ERR_CUDA.
+ * ---------------------------------------------------------------------------------- */
+SSD_API size_t ssd_prefill_workspace_size(int b, int T, int H, int P, int N, int G, int chunk,
+                                  int io_dtype);
+
+SSD_API int ssd_prefill(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype,
+                const void* x, const float* dt, const float* A, const void* B,
+                const void* C, const float* D, const float* h0, void* y, float* h_final,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Cached decode step  ([CF-SSD] O(1) caching section)
+ *
+ * One token for every (layer, sequence) pair, all layers in one launch.  With
+ * Dc = H*P + 2*G*N conv channels ordered [x (H*P) | B (G*N) | C (G*N)]:
+ *   h          [layers][b][H][P][N]   fp32, updated IN PLACE
+ *   conv_state [layers][b][Dc][k-1]   fp32, updated IN PLACE (oldest input first)
+ *   xbc        [layers][b][Dc]        io dtype: this token's pre-conv inputs
+ *   dt         [layers][b][H]         fp32 (positive)
+ *   A, D       [layers][H]            fp32
+ *   conv_w     [layers][Dc][k]        fp32: tap i multiplies window[i], where window =
+ *                                     [conv_state[..][0..k-2], xbc] (tap k-1 = current)
+ *   conv_b     [layers][Dc]           fp32
+ *   y          [layers][b][H][P]      io dtype (output)
+ * Per pair: u = act(conv(window) + bias); conv_state <- window[1..k-1];
+ * x, Bv, Cv = split(u); per head: h = exp(dt*A) h + dt * x Bv^T; y = h Cv + D x.
+ * act is SSD_ACT_NONE or SSD_ACT_SILU; kconv must be 4.  The workspace (see
+ * ssd_decode_workspace_size) holds per-(layer, sequence, group) arrival counters that
+ * the call zero-fills itself; calls sharing one workspace must be stream-ordered.
+ * Errors: as for ssd_prefill.
+ * ---------------------------------------------------------------------------------- */
+SSD_API size_t ssd_decode_workspace_size(int layers, int b, int G);
+
+SSD_API int ssd_decode_step(int layers, int b, int H, int P, int N, int G, int kconv, int act,
+                    int io_dtype, float* h, float* conv_state, const void* xbc,
+                    const float* dt, const float* A, const float* D, const float* conv_w,
+                    const float* conv_b, void* y, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * On-device decode loop  ([CF-SSD] "Compiled on-device loops")
+ *
+ * A plan records n_steps decode steps as one CUDA graph (a counter reset, then n_steps
+ * dependent step kernels) so that a launch runs every step with no host involvement.
+ * Step t of a launch (t = 0 .. n_steps-1, restarting at 0 on every launch) reads
+ * xbc_ring[t % ring] ([ring][layers][b][Dc]) and
+ * dt_ring[t % ring] ([ring][layers][b][H]) and writes y_ring[t % ring]
+ * ([ring][layers][b][H][P]); h and conv_state are carried in place from step to step.
+ * The plan keeps every pointer it was given; the caller keeps them alive and unmoved
+ * until ssd_decode_plan_destroy.  A plan may be launched any number of times (each
+ * launch continues from the current h / conv_state).  Plans are not thread-safe.
+ * ---------------------------------------------------------------------------------- */
+typedef struct ssd_decode_plan ssd_decode_plan;
+
+SSD_API int ssd_decode_plan_create(ssd_decode_plan** plan, int layers, int b, int H, int P, int N,
+                           int G, int kconv, int act, int io_dtype, float* h,
+                           float* conv_state, const void* xbc_ring, const float* dt_ring,
+                           int ring, const float* A, const float* D, const float* conv_w,
+                           const float* conv_b, void* y_ring, int n_steps, void* workspace,
+                           size_t workspace_bytes);
+
+SSD_API int ssd_decode_plan_launch(ssd_decode_plan* plan, void* stream);
+
+SSD_API int ssd_decode_plan_destroy(ssd_decode_plan* plan);
+
+/* ------------------------------------------------------------------------------------
+ * Measurement hooks (no counterpart on the pages; used by the benchmark)
+ *
+ * ssd_launch_count: total number of kernels this library has enqueued in this process
+ * (a decode plan launch counts its n_steps step kernels; memsets are not counted).
+ * ssd_profile_begin: from now on, every kernel launch is bracketed by a pair of CUDA
+ * events recorded on the launching stream (at most 65536 launches are kept).
+ * ssd_profile_end: waits for the recorded events, stops recording and reports per
+ * kernel name the number of launches and the summed event time in milliseconds, in
+ * first-launch order.  Returns the number of entries written (<= max_entries) or a
+ * negative ssd_status on failure.  Not thread-safe; kernels inside a decode plan are
+ * not bracketed (the plan launch as a whole is, under the name "decode_plan").
+ * ---------------------------------------------------------------------------------- */
+typedef struct {
+    char name[48];
+    int launches;
+    double total_ms;
+} ssd_kernel_time;
+
+SSD_API uint64_t ssd_launch_count(void);
+SSD_API int ssd_profile_begin(void);
+SSD_API int ssd_profile_end(ssd_kernel_time* out, int max_entries);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_B200_H_ */

@@ -91,7 +91,7 @@ def make_prefill(b, T, H, P, N, G, L, dtype="bf16", h0_std=0.0, seed=0,
     ``dt_scale`` multiplies dt after the draw (1.0 = the recipe); tests use it to
     build strong- or weak-decay edge cases.
     """
-    assert H % G == 0 and T % L == 0
+    assert H % G == 0
     rng = np.random.default_rng(seed)
     A, dt_bias = head_params(rng, H)
     z = rng.standard_normal((b, T, H), dtype=np.float32)
@@ -159,16 +159,41 @@ def make_decode(layers, b, H, P, N, G, k=4, ring=8, seed=3, h_std=0.1,
     """
     rng = np.random.default_rng(seed)
     Dc = H * P + 2 * G * N
+    A, D, conv_w, conv_b, dt_bias = _decode_params(rng, layers, H, P, N, G, k)
+    h = (rng.standard_normal((layers, b, H, P, N), dtype=np.float32) * np.float32(h_std)).astype(np.float32)
+    cs = (rng.standard_normal((layers, b, Dc, k - 1), dtype=np.float32) * np.float32(conv_state_std)).astype(np.float32)
+    xbc, bits = bf16_round(rng.standard_normal((ring, layers, b, Dc), dtype=np.float32))
+    z = rng.standard_normal((ring, layers, b, H), dtype=np.float32).astype(np.float64)
+    dt = _softplus(0.5 * z + dt_bias[None, :, None, :]).astype(np.float32)
+    return DecodeCase(layers, b, H, P, N, G, k, ring, A, D, conv_w, conv_b, h, cs, xbc, bits, dt)
+
+
+def _decode_params(rng, layers, H, P, N, G, k):
+    Dc = H * P + 2 * G * N
     A = np.empty((layers, H), np.float32)
     dt_bias = np.empty((layers, H), np.float64)
     for l in range(layers):
         A[l], dt_bias[l] = head_params(rng, H)
     conv_w = rng.uniform(-0.5, 0.5, size=(layers, Dc, k)).astype(np.float32)
     conv_b = rng.uniform(-0.5, 0.5, size=(layers, Dc)).astype(np.float32)
-    h = (rng.standard_normal((layers, b, H, P, N), dtype=np.float32) * np.float32(h_std)).astype(np.float32)
-    cs = (rng.standard_normal((layers, b, Dc, k - 1), dtype=np.float32) * np.float32(conv_state_std)).astype(np.float32)
-    xbc, bits = bf16_round(rng.standard_normal((ring, layers, b, Dc), dtype=np.float32))
-    z = rng.standard_normal((ring, layers, b, H), dtype=np.float32).astype(np.float64)
-    dt = _softplus(0.5 * z + dt_bias[None, :, None, :]).astype(np.float32)
     D = np.ones((layers, H), np.float32)
-    return DecodeCase(layers, b, H, P, N, G, k, ring, A, D, conv_w, conv_b, h, cs, xbc, bits, dt)
+    return A, D, conv_w, conv_b, dt_bias
+
+
+def make_decode_params(layers, H, P, N, G, k=4, seed=3):
+    """Per-layer A, D, conv weights/bias and dt_bias: the first draws of make_decode."""
+    return _decode_params(np.random.default_rng(seed), layers, H, P, N, G, k)
+
+
+def make_decode_ring_device(ring, layers, b, H, P, N, G, dt_bias, seed, device):
+    """Large decode step-input rings drawn on the device with a seeded torch generator
+    (same distributions as make_decode): xbc ~ N(0,1) in bf16, dt = softplus(0.5 z +
+    dt_bias).  Used where host generation of gigabytes would dominate the run."""
+    import torch
+    gen = torch.Generator(device=device).manual_seed(seed)
+    Dc = H * P + 2 * G * N
+    xbc = torch.randn((ring, layers, b, Dc), generator=gen, device=device).to(torch.bfloat16)
+    z = torch.randn((ring, layers, b, H), generator=gen, device=device)
+    bias = torch.as_tensor(dt_bias, dtype=torch.float32, device=device)[None, :, None, :]
+    dt = torch.nn.functional.softplus(0.5 * z + bias).contiguous()
+    return xbc, dt

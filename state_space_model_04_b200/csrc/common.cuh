@@ -1,0 +1,55 @@
+// common.cuh -- small shared helpers for the sm_100a SSD kernels (no method arithmetic
+// beyond type conversion lives here).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/ssd.h"
+
+namespace ssd {
+
+// Records a detail string for ssd_last_error() and returns the status unchanged.
+int set_error(int status, const char* fmt, ...);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Load one io element as float.
+__device__ __forceinline__ float load_io(const float* p, size_t i) { return p[i]; }
+__device__ __forceinline__ float load_io(const __nv_bfloat16* p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_io(float* p, size_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void store_io(__nv_bfloat16* p, size_t i, float v) {
+    p[i] = __float2bfloat16_rn(v);
+}
+
+// Map a CUDA error to a status with detail.
+int cuda_status(cudaError_t e, const char* where);
+
+// Launch accounting and optional per-kernel event timing (see ssd_profile_begin).
+void count_launches(uint64_t n);
+void prof_start(const char* name, cudaStream_t s);  // no-op unless profiling
+void prof_stop(cudaStream_t s);
+
+// Brackets one launch: counts it and, when profiling, records events around it.
+struct LaunchScope {
+    cudaStream_t s;
+    LaunchScope(const char* name, cudaStream_t st, uint64_t n = 1) : s(st) {
+        count_launches(n);
+        prof_start(name, st);
+    }
+    ~LaunchScope() { prof_stop(s); }
+};
+
+}  // namespace ssd
+
+#define SSD_CUDA_TRY(expr)                                                   \
+    do {                                                                     \
+        cudaError_t e_ = (expr);                                             \
+        if (e_ != cudaSuccess) return ::ssd::cuda_status(e_, #expr);         \
+    } while (0)

@@ -1,0 +1,263 @@
+"""Python binding of libssd_b200.so (argument marshalling only).
+
+Every step of the SSD prefill and decode runs in the library's sm_100a kernels; this
+module checks tensor dtypes/devices/shapes, allocates outputs and workspaces with torch
+(device memory and streams are the only things torch provides) and forwards raw
+pointers to the C ABI declared in include/ssd.h.  There is no CPU fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssd_b200.so")
+
+SSD_OK = 0
+SSD_F32, SSD_BF16 = 0, 1
+SSD_ACT_NONE, SSD_ACT_SILU = 0, 1
+
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+_vp = ctypes.c_void_p
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__("%s failed: status %d (%s) %s" % (where, status, status_string(status), detail))
+        self.status = status
+
+
+class _KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int), ("total_ms", ctypes.c_double)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libssd_b200.so; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libssd_b200.so is not built: run `python -m state_space_model_04_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.ssd_version.restype = _i
+        L.ssd_status_string.argtypes = [_i]
+        L.ssd_status_string.restype = ctypes.c_char_p
+        L.ssd_last_error.restype = ctypes.c_char_p
+        L.ssd_prefill_workspace_size.argtypes = [_i] * 8
+        L.ssd_prefill_workspace_size.restype = _sz
+        L.ssd_prefill.argtypes = [_i] * 8 + [_vp] * 10 + [_sz, _vp]
+        L.ssd_prefill.restype = _i
+        L.ssd_decode_workspace_size.argtypes = [_i] * 3
+        L.ssd_decode_workspace_size.restype = _sz
+        L.ssd_decode_step.argtypes = [_i] * 9 + [_vp] * 10 + [_sz, _vp]
+        L.ssd_decode_step.restype = _i
+        L.ssd_decode_plan_create.argtypes = [ctypes.POINTER(_vp)] + [_i] * 9 + [_vp] * 4 + [_i] + [_vp] * 5 + [_i, _vp, _sz]
+        L.ssd_decode_plan_create.restype = _i
+        L.ssd_decode_plan_launch.argtypes = [_vp, _vp]
+        L.ssd_decode_plan_launch.restype = _i
+        L.ssd_decode_plan_destroy.argtypes = [_vp]
+        L.ssd_decode_plan_destroy.restype = _i
+        L.ssd_launch_count.restype = ctypes.c_uint64
+        L.ssd_profile_begin.restype = _i
+        L.ssd_profile_end.argtypes = [ctypes.POINTER(_KernelTime), _i]
+        L.ssd_profile_end.restype = _i
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().ssd_status_string(int(status)).decode()
+
+
+def last_error() -> str:
+    return lib().ssd_last_error().decode()
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued in this process (decode plans count their steps)."""
+    return int(lib().ssd_launch_count())
+
+
+def profile_begin():
+    """Start bracketing every library kernel launch with CUDA events on its stream."""
+    _check(lib().ssd_profile_begin(), "ssd_profile_begin")
+
+
+def profile_end(max_entries=64):
+    """Stop and return {kernel name: (launches, summed event milliseconds)}."""
+    buf = (_KernelTime * max_entries)()
+    n = lib().ssd_profile_end(buf, max_entries)
+    if n < 0:
+        _check(-n, "ssd_profile_end")
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms) for i in range(n)}
+
+
+def _check(status: int, where: str):
+    if status != SSD_OK:
+        raise SSDError(status, where, last_error())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _io(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SSD_BF16
+    if t.dtype == torch.float32:
+        return SSD_F32
+    raise TypeError("io tensors must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _need(t, name, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor (no CPU path exists)" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    return t
+
+
+def prefill_workspace_size(b, T, H, P, N, G, chunk, io_dtype) -> int:
+    return int(lib().ssd_prefill_workspace_size(b, T, H, P, N, G, chunk, io_dtype))
+
+
+def prefill(x, dt, A, B, C, D, chunk=256, h0=None, y=None, h_final=None, workspace=None,
+            want_final=True, stream=None):
+    """Chunked SSD prefill.  Shapes: x [b,T,H,P], dt [b,T,H] f32, A [H] f32,
+    B/C [b,T,G,N], D [H] f32, h0 [b,H,P,N] f32 or None.  Returns (y, h_final)."""
+    _need(x, "x")
+    io = _io(x)
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    _need(dt, "dt", torch.float32, (b, T, H))
+    _need(A, "A", torch.float32, (H,))
+    _need(D, "D", torch.float32, (H,))
+    _need(B, "B", x.dtype, (b, T, G, N))
+    _need(C, "C", x.dtype, (b, T, G, N))
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (b, H, P, N))
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", x.dtype, x.shape)
+    if h_final is None and want_final:
+        h_final = torch.empty((b, H, P, N), dtype=torch.float32, device=x.device)
+    if h_final is not None:
+        _need(h_final, "h_final", torch.float32, (b, H, P, N))
+    need = prefill_workspace_size(b, T, H, P, N, G, chunk, io)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().ssd_prefill(b, T, H, P, N, G, int(chunk), io, _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                           _ptr(C), _ptr(D), _ptr(h0), _ptr(y), _ptr(h_final), _ptr(workspace),
+                           ws_bytes, _stream(stream))
+    _check(st, "ssd_prefill")
+    return y, h_final
+
+
+def decode_workspace_size(layers, b, G) -> int:
+    return int(lib().ssd_decode_workspace_size(layers, b, G))
+
+
+def _decode_shapes(h, conv_state, A, D, conv_w, conv_b, G):
+    _need(h, "h", torch.float32)
+    layers, b, H, P, N = h.shape
+    k = conv_w.shape[-1]
+    Dc = H * P + 2 * G * N
+    _need(conv_state, "conv_state", torch.float32, (layers, b, Dc, k - 1))
+    _need(A, "A", torch.float32, (layers, H))
+    _need(D, "D", torch.float32, (layers, H))
+    _need(conv_w, "conv_w", torch.float32, (layers, Dc, k))
+    _need(conv_b, "conv_b", torch.float32, (layers, Dc))
+    return layers, b, H, P, N, k, Dc
+
+
+def decode_step(h, conv_state, xbc, dt, A, D, conv_w, conv_b, G=1, act=SSD_ACT_SILU, y=None,
+                workspace=None, stream=None):
+    """One decode step for all layers; h and conv_state are updated in place.  Returns y."""
+    layers, b, H, P, N, k, Dc = _decode_shapes(h, conv_state, A, D, conv_w, conv_b, G)
+    _need(xbc, "xbc", None, (layers, b, Dc))
+    io = _io(xbc)
+    _need(dt, "dt", torch.float32, (layers, b, H))
+    if y is None:
+        y = torch.empty((layers, b, H, P), dtype=xbc.dtype, device=h.device)
+    _need(y, "y", xbc.dtype, (layers, b, H, P))
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_size(layers, b, G), dtype=torch.uint8, device=h.device)
+    st = lib().ssd_decode_step(layers, b, H, P, N, G, k, act, io, _ptr(h), _ptr(conv_state), _ptr(xbc),
+                               _ptr(dt), _ptr(A), _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(y),
+                               _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "ssd_decode_step")
+    return y
+
+
+class DecodePlan:
+    """n_steps decode steps recorded once as a CUDA graph; launch() runs them all on the
+    device with no host round trip.  Step t reads xbc_ring[t % ring], dt_ring[t % ring]
+    and writes y_ring[t % ring].  The plan holds references to every tensor it uses."""
+
+    def __init__(self, h, conv_state, xbc_ring, dt_ring, A, D, conv_w, conv_b, n_steps, G=1,
+                 act=SSD_ACT_SILU, y_ring=None):
+        layers, b, H, P, N, k, Dc = _decode_shapes(h, conv_state, A, D, conv_w, conv_b, G)
+        ring = xbc_ring.shape[0]
+        _need(xbc_ring, "xbc_ring", None, (ring, layers, b, Dc))
+        io = _io(xbc_ring)
+        _need(dt_ring, "dt_ring", torch.float32, (ring, layers, b, H))
+        if y_ring is None:
+            y_ring = torch.empty((ring, layers, b, H, P), dtype=xbc_ring.dtype, device=h.device)
+        _need(y_ring, "y_ring", xbc_ring.dtype, (ring, layers, b, H, P))
+        self.workspace = torch.empty(decode_workspace_size(layers, b, G), dtype=torch.uint8, device=h.device)
+        self._keep = (h, conv_state, xbc_ring, dt_ring, A, D, conv_w, conv_b, y_ring)
+        self.y_ring = y_ring
+        self.n_steps = n_steps
+        handle = ctypes.c_void_p()
+        st = lib().ssd_decode_plan_create(ctypes.byref(handle), layers, b, H, P, N, G, k, act, io,
+                                          _ptr(h), _ptr(conv_state), _ptr(xbc_ring), _ptr(dt_ring), ring,
+                                          _ptr(A), _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(y_ring),
+                                          int(n_steps), _ptr(self.workspace), self.workspace.numel())
+        _check(st, "ssd_decode_plan_create")
+        self._h = handle
+
+    def launch(self, stream=None):
+        if self._h is None:
+            raise RuntimeError("plan destroyed")
+        _check(lib().ssd_decode_plan_launch(self._h, _stream(stream)), "ssd_decode_plan_launch")
+        return self.y_ring
+
+    def close(self):
+        if getattr(self, "_h", None) is not None:
+            _check(lib().ssd_decode_plan_destroy(self._h), "ssd_decode_plan_destroy")
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def decode_loop(h, conv_state, xbc_ring, dt_ring, A, D, conv_w, conv_b, n_steps, G=1,
+                act=SSD_ACT_SILU, stream=None):
+    """Run n_steps decode steps as one graph launch (plan built, launched, released)."""
+    plan = DecodePlan(h, conv_state, xbc_ring, dt_ring, A, D, conv_w, conv_b, n_steps, G, act)
+    y = plan.launch(stream)
+    torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+    plan.close()
+    return y

@@ -1,0 +1,158 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every entry
+point include/ssd.h declares, and rejects bad arguments with the documented status
+before anything is enqueued.  Pointers here are fake but 16-byte aligned addresses; a
+validation failure must return before they are ever dereferenced or passed to CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import state_space_model_04_b200 as ssd
+from state_space_model_04_b200 import ssd as binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, INVALID, UNSUP, CUDA, TIMEOUT, WS, INTERNAL = range(7)
+
+pytestmark = pytest.mark.skipif(not os.path.exists(binding.LIB_PATH), reason="library not built")
+
+
+def _declared():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"SSD_API\s+[\w\s\*]+?\b(ssd_\w+)\s*\(", txt)
+    return names
+
+
+def test_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 10
+    L = ssd.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_status_strings():
+    L = ssd.lib()
+    assert L.ssd_version() >= 100
+    for s in range(7):
+        assert ssd.status_string(s).startswith("SSD_")
+    assert "unknown" in ssd.status_string(99)
+
+
+# fake, aligned, distinct device addresses (never dereferenced: validation fails first)
+def _fake(n):
+    return [ctypes.c_void_p(0x10000000 + 0x1000000 * i) for i in range(n)]
+
+
+def _prefill(b=1, T=512, H=4, P=64, N=64, G=1, chunk=256, io=1, ptrs=None, ws_bytes=1 << 30,
+             h0=None, hf=None):
+    L = ssd.lib()
+    x, dt, A, B, C, D, y, ws = ptrs or _fake(8)
+    return L.ssd_prefill(b, T, H, P, N, G, chunk, io, x, dt, A, B, C, D, h0, y, hf, ws,
+                         ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(chunk=100), INVALID), (dict(chunk=32), INVALID), (dict(io=7), INVALID),
+    (dict(H=6, G=4), INVALID), (dict(b=-1), INVALID), (dict(T=-5), INVALID), (dict(N=0), INVALID),
+    (dict(P=32), UNSUP), (dict(N=96), UNSUP), (dict(b=70000), UNSUP),
+    (dict(ws_bytes=16), WS),
+])
+def test_prefill_rejects(kw, status):
+    assert _prefill(**kw) == status
+    assert ssd.last_error() != ""
+
+
+def test_prefill_null_and_misaligned_pointers():
+    for i in range(7):  # x, dt, A, B, C, D, y
+        p = _fake(8)
+        p[i] = None
+        assert _prefill(ptrs=p) == INVALID, i
+        p = _fake(8)
+        p[i] = ctypes.c_void_p(p[i].value + 4)
+        assert _prefill(ptrs=p) == INVALID, i
+    p = _fake(8)
+    p[7] = None
+    assert _prefill(ptrs=p) == WS
+
+
+def test_prefill_rejects_aliasing():
+    p = _fake(8)
+    p[6] = p[0]  # y == x
+    assert _prefill(ptrs=p) == INVALID
+    p = _fake(8)
+    hf = ctypes.c_void_p(p[0].value)  # h_final overlaps x
+    assert _prefill(ptrs=p, hf=hf) == INVALID
+    h0 = ctypes.c_void_p(0x7000000000)
+    hf = ctypes.c_void_p(0x7000000000 + 4096)  # partial overlap of h0 / h_final
+    assert _prefill(ptrs=_fake(8), h0=h0, hf=hf) == INVALID
+
+
+def test_prefill_empty_batch_is_noop():
+    assert _prefill(b=0) == OK
+    assert _prefill(T=0) == OK  # no h_final requested: nothing to do, no CUDA call
+
+
+def test_workspace_queries():
+    assert ssd.prefill_workspace_size(1, 512, 4, 64, 64, 1, 256, 0) > 0
+    assert ssd.prefill_workspace_size(8, 4096, 80, 64, 128, 1, 256, 1) > 0
+    assert ssd.prefill_workspace_size(1, 512, 4, 64, 64, 1, 100, 0) == 0  # invalid chunk
+    assert ssd.prefill_workspace_size(0, 512, 4, 64, 64, 1, 256, 0) == 0
+    assert ssd.decode_workspace_size(64, 32, 1) >= 64 * 32 * 4
+    assert ssd.decode_workspace_size(0, 1, 1) == 0
+
+
+def _decode(layers=2, b=1, H=4, P=64, N=128, G=1, k=4, act=1, io=1, ptrs=None, ws_bytes=1 << 20):
+    L = ssd.lib()
+    h, cs, xbc, dt, A, D, w, bb, y, ws = ptrs or _fake(10)
+    return L.ssd_decode_step(layers, b, H, P, N, G, k, act, io, h, cs, xbc, dt, A, D, w, bb, y, ws,
+                             ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(act=3), INVALID), (dict(io=2), INVALID), (dict(H=5, G=2), INVALID), (dict(k=0), INVALID),
+    (dict(k=3), UNSUP), (dict(P=128), UNSUP), (dict(N=32), UNSUP), (dict(layers=-1), INVALID),
+    (dict(ws_bytes=0), WS),
+])
+def test_decode_rejects(kw, status):
+    assert _decode(**kw) == status
+
+
+def test_decode_null_aliasing_and_empty():
+    for i in range(10):
+        p = _fake(10)
+        p[i] = None
+        assert _decode(ptrs=p) in (INVALID, WS), i
+    p = _fake(10)
+    p[8] = p[0]  # y aliases h
+    assert _decode(ptrs=p) == INVALID
+    assert _decode(b=0) == OK
+    assert _decode(layers=0) == OK
+
+
+def test_decode_plan_rejects():
+    L = ssd.lib()
+    handle = ctypes.c_void_p()
+    f = _fake(10)
+    # ring = 0
+    st = L.ssd_decode_plan_create(ctypes.byref(handle), 1, 1, 4, 64, 128, 1, 4, 1, 1, f[0], f[1], f[2],
+                                  f[3], 0, f[4], f[5], f[6], f[7], f[8], 8, f[9], 1 << 20)
+    assert st == INVALID and not handle.value
+    st = L.ssd_decode_plan_create(ctypes.byref(handle), 1, 1, 4, 64, 128, 1, 4, 1, 1, f[0], f[1], f[2],
+                                  f[3], 2, f[4], f[5], f[6], f[7], f[8], -1, f[9], 1 << 20)
+    assert st == INVALID
+    assert L.ssd_decode_plan_create(None, 1, 1, 4, 64, 128, 1, 4, 1, 1, f[0], f[1], f[2], f[3], 2,
+                                    f[4], f[5], f[6], f[7], f[8], 8, f[9], 1 << 20) == INVALID
+    assert L.ssd_decode_plan_launch(None, None) == INVALID
+    assert L.ssd_decode_plan_destroy(None) == OK
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 64, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        ssd.prefill(x, torch.zeros(1, 64, 4), torch.zeros(4), torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16),
+                    torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16), torch.zeros(4))

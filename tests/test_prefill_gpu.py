@@ -1,0 +1,186 @@
+"""GPU parity of ssd_prefill against the fp64 oracle (called through the C ABI binding).
+
+Covers: the tiny fp32 configuration (fp32 gate), small bf16/fp32 problems that span
+several chunks and a ragged tail, every chunk length, grouped B/C, the 130M-layer
+configuration in full, the 2.7B-layer and long-context configurations at full size on
+sampled (sequence, head) pairs, and the invariants of "Compiler-First State Space
+Duality ..." (chunking changes nothing, batch invariance, causality, the prefill's final
+state resumes the sequence).  Edge cases: T = 0, b = 0, T = 1, T < chunk, strong decay,
+h0 aliasing h_final.
+"""
+import numpy as np
+import pytest
+import torch
+
+from ssd_inputs import make_config, make_prefill
+from tests.helpers import check, oracle_subset, prefill_inputs, run_prefill
+
+pytestmark = pytest.mark.gpu
+
+ssd = pytest.importorskip("state_space_model_04_b200")
+
+
+def _np(t):
+    return t.float().cpu().numpy()
+
+
+def _full_check(case, chunk=None, nthreads=0):
+    y, hf, _ = run_prefill(ssd, case, chunk)
+    y_ref, hf_ref = oracle_subset(case, range(case.b), range(case.H), nthreads)
+    e1 = check(_np(y), y_ref, case.dtype, "y")
+    e2 = check(_np(hf), hf_ref, case.dtype, "h_final")
+    return e1, e2
+
+
+def test_tiny_f32_config():
+    """The fp32 configuration (b=1, T=512, H=4, P=64, N=64) at the fp32 gate."""
+    _full_check(make_config("tiny_f32"))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("shape", [
+    # b, T, H, N, G, L  -- several chunks, ragged tails, groups, every chunk length
+    (2, 600, 4, 128, 1, 256),
+    (1, 384, 6, 64, 3, 128),
+    (1, 200, 2, 128, 2, 64),
+    (3, 129, 2, 64, 1, 128),
+    (1, 1000, 8, 128, 4, 256),
+])
+def test_small_cases(dtype, shape):
+    b, T, H, N, G, L = shape
+    case = make_prefill(b, T, H, 64, N, G, L, dtype=dtype, h0_std=0.1, seed=sum(shape))
+    _full_check(case)
+
+
+def test_130m_layer_config_full():
+    """b=1, T=4096, H=24, N=128, L=256, bf16: every output against the oracle."""
+    _full_check(make_config("mamba2_130m_layer"))
+
+
+def test_2p7b_layer_config_sampled():
+    """b=8, T=4096, H=80, N=128, L=256, bf16, h0 ~ N(0, 0.1): full-size launch, sequences
+    {0, 7} x heads {0, 41, 79} against the oracle."""
+    case = make_config("mamba2_2p7b_layer")
+    y, hf, _ = run_prefill(ssd, case)
+    seqs, heads = [0, 7], [0, 41, 79]
+    y_ref, hf_ref = oracle_subset(case, seqs, heads)
+    ys = y[seqs][:, :, heads]
+    hs = hf[seqs][:, heads]
+    check(_np(ys), y_ref, "bf16", "y")
+    check(_np(hs), hf_ref, "bf16", "h_final")
+    assert torch.isfinite(y.float()).all() and torch.isfinite(hf).all()
+
+
+@pytest.mark.parametrize("L", [64, 128, 256])
+def test_long_context_sampled(L):
+    """b=1, T=65536, H=80, G=8 at each chunk length: heads {0, 45, 79} (groups 0, 5, 7)."""
+    case = make_config("long_context_L%d" % L)
+    y, hf, _ = run_prefill(ssd, case)
+    heads = [0, 45, 79]
+    y_ref, hf_ref = oracle_subset(case, [0], heads)
+    check(_np(y[:, :, heads]), y_ref, "bf16", "y")
+    check(_np(hf[:, heads]), hf_ref, "bf16", "h_final")
+    assert torch.isfinite(y.float()).all()
+
+
+# ------------------------------------------------------------------ invariants
+def test_deterministic_bitwise():
+    case = make_prefill(2, 700, 4, 64, 128, 2, 256, "bf16", h0_std=0.1, seed=5)
+    y1, h1, _ = run_prefill(ssd, case)
+    y2, h2, _ = run_prefill(ssd, case)
+    assert torch.equal(y1, y2) and torch.equal(h1, h2)
+
+
+def test_batch_invariance_bitwise():
+    case = make_prefill(3, 520, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=6)
+    y, hf, t = run_prefill(ssd, case)
+    y1, h1 = ssd.prefill(t["x"][1:2].contiguous(), t["dt"][1:2].contiguous(), t["A"], t["B"][1:2].contiguous(),
+                         t["C"][1:2].contiguous(), t["D"], chunk=256, h0=t["h0"][1:2].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(y[1:2], y1) and torch.equal(hf[1:2], h1)
+
+
+def test_causality_bitwise():
+    case = make_prefill(1, 768, 4, 64, 128, 1, 256, "bf16", seed=7)
+    y, _, t = run_prefill(ssd, case)
+    x2 = t["x"].clone()
+    x2[:, 400] += 1.0
+    y2, _ = ssd.prefill(x2, t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=256)
+    torch.cuda.synchronize()
+    assert torch.equal(y[:, :400], y2[:, :400])
+    assert not torch.equal(y[:, 400:], y2[:, 400:])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_split_resume(dtype):
+    """prefill(T1+T2) == prefill(T2, h0 = h_final(prefill(T1))): prefill fills the cache."""
+    case = make_prefill(2, 1024, 4, 64, 128, 1, 256, dtype, h0_std=0.1, seed=8)
+    y, hf, t = run_prefill(ssd, case)
+    s = 384
+    y1, h1 = ssd.prefill(t["x"][:, :s].contiguous(), t["dt"][:, :s].contiguous(), t["A"], t["B"][:, :s].contiguous(),
+                         t["C"][:, :s].contiguous(), t["D"], chunk=256, h0=t["h0"])
+    y2, h2 = ssd.prefill(t["x"][:, s:].contiguous(), t["dt"][:, s:].contiguous(), t["A"], t["B"][:, s:].contiguous(),
+                         t["C"][:, s:].contiguous(), t["D"], chunk=256, h0=h1)
+    torch.cuda.synchronize()
+    check(_np(torch.cat([y1, y2], 1)), _np(y), dtype, "y")
+    check(_np(h2), _np(hf), dtype, "h_final")
+
+
+def test_chunk_length_invariance():
+    case = make_prefill(1, 1024, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=9)
+    ys = [run_prefill(ssd, case, chunk=L)[0] for L in (64, 128, 256)]
+    for y in ys[:2]:
+        check(_np(y), _np(ys[2]), "bf16", "chunk invariance")
+
+
+# ------------------------------------------------------------------ edge cases
+def test_empty_sequence_passes_state_through():
+    case = make_prefill(2, 256, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=10)
+    t = prefill_inputs(case)
+    x0 = t["x"][:, :0].contiguous()
+    y, hf = ssd.prefill(x0, t["dt"][:, :0].contiguous(), t["A"], t["B"][:, :0].contiguous(),
+                        t["C"][:, :0].contiguous(), t["D"], chunk=256, h0=t["h0"])
+    torch.cuda.synchronize()
+    assert y.numel() == 0 and torch.equal(hf, t["h0"])
+    _, hz = ssd.prefill(x0, t["dt"][:, :0].contiguous(), t["A"], t["B"][:, :0].contiguous(),
+                        t["C"][:, :0].contiguous(), t["D"], chunk=256)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(hz) == 0
+
+
+def test_empty_batch():
+    case = make_prefill(1, 64, 2, 64, 64, 1, 64, "bf16", seed=11)
+    t = prefill_inputs(case)
+    y, hf = ssd.prefill(t["x"][:0].contiguous(), t["dt"][:0].contiguous(), t["A"], t["B"][:0].contiguous(),
+                        t["C"][:0].contiguous(), t["D"], chunk=64)
+    assert y.numel() == 0 and hf.numel() == 0
+
+
+@pytest.mark.parametrize("T", [1, 63, 255, 257])
+def test_short_and_ragged(T):
+    case = make_prefill(1, T, 3, 64, 128, 1, 1, "bf16", h0_std=0.1, seed=T)
+    _full_check(case, chunk=256 if T > 64 else 64)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_strong_decay(dtype):
+    """dt 50x the recipe: exp(cs) underflows within a chunk; results stay finite and exact."""
+    case = make_prefill(1, 512, 4, 64, 128, 1, 256, dtype, h0_std=0.1, seed=12, dt_scale=50.0)
+    _full_check(case)
+
+
+def test_weak_decay_long_memory():
+    """dt 0.01x the recipe: almost no decay, the state accumulates over the whole sequence."""
+    case = make_prefill(1, 2048, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=13, dt_scale=0.01)
+    _full_check(case)
+
+
+def test_in_place_state_resume():
+    """h_final may alias h0 exactly (in-place cache update)."""
+    case = make_prefill(1, 512, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=14)
+    y, hf, t = run_prefill(ssd, case)
+    h = t["h0"].clone()
+    y2, h2 = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=256, h0=h, h_final=h)
+    torch.cuda.synchronize()
+    assert h2.data_ptr() == h.data_ptr()
+    assert torch.equal(y2, y) and torch.equal(h, hf)
