@@ -133,6 +133,33 @@ SSD_API int ssd_decode_step(int layers, int b, int H, int P, int N, int G, int k
                     void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * Allocation-free decode step  (the paper has no counterpart: this is an integration
+ * entry point, not part of the method)
+ *
+ * For callers that cannot allocate device memory or hand the library a workspace: code
+ * that runs inside an engine's enqueue/plugin hook where the engine owns every byte of
+ * device memory, code recorded while a CUDA graph is being captured (cudaMalloc is not
+ * allowed then), and real-time serving loops that forbid allocation after start-up.
+ * Same arguments, semantics and errors as ssd_decode_step, without the workspace.  The
+ * scratch it needs (one 32-bit arrival counter per (layer, sequence, group)) lives in a
+ * file-scope device array of SSD_DECODE_NOALLOC_MAX_COUNTERS counters (256 KiB) that
+ * every GPU which loads the library keeps until the process exits; layers*b*G above
+ * that limit returns SSD_ERR_INVALID_ARG.  The first call on a device looks up the
+ * array's device address with that device current (cudaGetSymbolAddress), so make that
+ * first call before any stream capture.  Each call clears the counters it uses
+ * (cudaMemsetAsync on `stream`) and calls no cudaMalloc, cudaFree or allocating
+ * routine.  All calls on a device share the one array: calls that overlap on the GPU
+ * (unordered streams) race on it and corrupt each other's conv windows.
+ * ---------------------------------------------------------------------------------- */
+#define SSD_DECODE_NOALLOC_MAX_COUNTERS 65536
+
+SSD_API int ssd_decode_step_noalloc(int layers, int b, int H, int P, int N, int G, int kconv,
+                                    int act, int io_dtype, float* h, float* conv_state,
+                                    const void* xbc, const float* dt, const float* A,
+                                    const float* D, const float* conv_w, const float* conv_b,
+                                    void* y, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * On-device decode loop  ([CF-SSD] "Compiled on-device loops")
  *
  * A plan records n_steps decode steps as one CUDA graph (a counter reset, then n_steps

@@ -13,6 +13,7 @@ from .ssd import (  # noqa: F401
     SSDError,
     decode_loop,
     decode_step,
+    decode_step_noalloc,
     decode_workspace_size,
     last_error,
     launch_count,

@@ -32,6 +32,7 @@ int create_decode_plan(ssd_decode_plan** out, int layers, int b, int H, int N, i
                        void* ws);
 int launch_decode_plan(ssd_decode_plan* plan, cudaStream_t s);
 int destroy_decode_plan(ssd_decode_plan* plan);
+int decode_noalloc_scratch(void** ptr, size_t* bytes);
 
 static thread_local char g_detail[512];
 
@@ -291,6 +292,24 @@ int ssd_decode_step(int layers, int b, int H, int P, int N, int G, int kconv, in
             return set_error(SSD_ERR_INVALID_ARG, "an input overlaps h, conv_state or y");
     return launch_decode_step(layers, b, H, N, G, act, io_dtype, h, conv_state, xbc, dt, A, D, conv_w,
                               conv_b, y, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int ssd_decode_step_noalloc(int layers, int b, int H, int P, int N, int G, int kconv, int act,
+                            int io_dtype, float* h, float* conv_state, const void* xbc,
+                            const float* dt, const float* A, const float* D, const float* conv_w,
+                            const float* conv_b, void* y, void* stream) {
+    g_detail[0] = 0;
+    if (layers > 0 && b > 0 && G > 0 &&
+        (size_t)layers * (size_t)b * (size_t)G > (size_t)SSD_DECODE_NOALLOC_MAX_COUNTERS)
+        return set_error(SSD_ERR_INVALID_ARG,
+                         "layers*b*G = %zu exceeds the %d arrival counters of the allocation-free decode step",
+                         (size_t)layers * b * G, SSD_DECODE_NOALLOC_MAX_COUNTERS);
+    void* scratch = nullptr;
+    size_t cap = 0;
+    if (layers > 0 && b > 0) SSD_CHECK(decode_noalloc_scratch(&scratch, &cap));
+    // the library's own scratch stands in for the caller workspace of ssd_decode_step
+    return ssd_decode_step(layers, b, H, P, N, G, kconv, act, io_dtype, h, conv_state, xbc, dt, A, D,
+                           conv_w, conv_b, y, scratch, cap, stream);
 }
 
 int ssd_decode_plan_create(ssd_decode_plan** plan, int layers, int b, int H, int P, int N, int G,

@@ -16,6 +16,7 @@
 // finish (an arrival counter, no waiting) writes the shifted window back.
 #include "common.cuh"
 
+#include <mutex>
 #include <vector>
 
 namespace ssd {
@@ -284,6 +285,37 @@ int destroy_decode_plan(ssd_decode_plan* plan) {
     delete plan;
     if (e1 != cudaSuccess) return cuda_status(e1, "cudaGraphExecDestroy");
     if (e2 != cudaSuccess) return cuda_status(e2, "cudaGraphDestroy");
+    return SSD_OK;
+}
+
+}  // namespace ssd
+
+// ---------------------------------------------------------------------------------------
+// Scratch for the allocation-free decode step: the arrival counters live in a file-scope
+// device array instead of a caller workspace.  Every GPU that loads the library holds it
+// (SSD_DECODE_NOALLOC_MAX_COUNTERS x 4 bytes) until the process exits.  In host code the
+// name g_noalloc_arrivals is only a stand-in; its device address is looked up per device.
+static __device__ __align__(256) unsigned int g_noalloc_arrivals[SSD_DECODE_NOALLOC_MAX_COUNTERS];
+
+namespace ssd {
+
+// Device address and size of the scratch array on the current device.  The first call on
+// a device resolves the address with that device current and caches it.
+int decode_noalloc_scratch(void** ptr, size_t* bytes) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    SSD_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return set_error(SSD_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kMaxDevices - 1);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        SSD_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_arrivals));
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    *bytes = sizeof(g_noalloc_arrivals);
     return SSD_OK;
 }
 

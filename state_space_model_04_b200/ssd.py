@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_decode_plan_launch.restype = _i
         L.ssd_decode_plan_destroy.argtypes = [_vp]
         L.ssd_decode_plan_destroy.restype = _i
+        L.ssd_decode_step_noalloc.argtypes = [_i] * 9 + [_vp] * 10
+        L.ssd_decode_step_noalloc.restype = _i
         L.ssd_launch_count.restype = ctypes.c_uint64
         L.ssd_profile_begin.restype = _i
         L.ssd_profile_end.argtypes = [ctypes.POINTER(_KernelTime), _i]
@@ -205,6 +207,23 @@ def decode_step(h, conv_state, xbc, dt, A, D, conv_w, conv_b, G=1, act=SSD_ACT_S
                                _ptr(dt), _ptr(A), _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(y),
                                _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "ssd_decode_step")
+    return y
+
+
+def decode_step_noalloc(h, conv_state, xbc, dt, A, D, conv_w, conv_b, y, G=1, act=SSD_ACT_SILU,
+                        stream=None):
+    """decode_step through ssd_decode_step_noalloc: no workspace, and the caller passes
+    the output y, so nothing is allocated on this path (for callers that cannot allocate
+    device memory).  Calls that overlap on the GPU race on the library's shared scratch."""
+    layers, b, H, P, N, k, Dc = _decode_shapes(h, conv_state, A, D, conv_w, conv_b, G)
+    _need(xbc, "xbc", None, (layers, b, Dc))
+    io = _io(xbc)
+    _need(dt, "dt", torch.float32, (layers, b, H))
+    _need(y, "y", xbc.dtype, (layers, b, H, P))
+    st = lib().ssd_decode_step_noalloc(layers, b, H, P, N, G, k, act, io, _ptr(h), _ptr(conv_state),
+                                       _ptr(xbc), _ptr(dt), _ptr(A), _ptr(D), _ptr(conv_w), _ptr(conv_b),
+                                       _ptr(y), _stream(stream))
+    _check(st, "ssd_decode_step_noalloc")
     return y
 
 
