@@ -231,6 +231,7 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- our arm
 def main():
+    global PB
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -239,6 +240,9 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024, help="timed decode steps at batch 1")
     ap.add_argument("--decode-batches", default="1,32")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-batch", type=int, default=PB,
+                    help="sequences per prefill step (default: the 2.7B-layer configuration's 8); "
+                         "smaller values are for profiling captures only")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -274,7 +278,8 @@ def main():
     stream = torch.cuda.current_stream()
 
     # ---------------- prefill inputs (seeded per rank: independent batches)
-    case = make_config("mamba2_2p7b_layer", seed=2 + 1000 * rank)
+    PB = args.prefill_batch
+    case = make_config("mamba2_2p7b_layer", seed=2 + 1000 * rank, b=PB)
     def bf(bits):
         return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
     host = {"x": bf(case.x_bits), "B": bf(case.B_bits), "C": bf(case.C_bits),

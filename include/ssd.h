@@ -88,9 +88,11 @@ SSD_API const char* ssd_last_error(void);
  * through the chunked dual form.  T need not be a multiple of `chunk`: the last chunk
  * is then shorter.  T == 0 or b == 0 is a no-op apart from h_final = h0 (or zeros).
  * chunk must be 64, 128 or 256.  x, B, C, dt, A, D must not alias y or h_final.
- * Arithmetic: SSD_BF16 inputs use bf16 tensor-core contractions (tcgen05) with fp32
- * accumulation, fp32 decay in log space and an fp32 running state; SSD_F32 inputs use
- * fp32 FMA with the prefix sums of dt*A kept in fp64 (no TF32 anywhere).
+ * Arithmetic: SSD_BF16 inputs with P == 64 and N == 128 run one fused tensor-core kernel
+ * (tcgen05 bf16 contractions, fp32 accumulation, fp32 decay in log space, fp32 running
+ * state kept on chip, 128-token blocks); other bf16 shapes and all SSD_F32 inputs run
+ * the four-kernel fp32-FMA path with the prefix sums of dt*A kept in fp64 (no TF32).
+ * The workspace's first 256 bytes hold a device status word (see ssd_prefill_check).
  * Errors: SSD_ERR_INVALID_ARG (null pointer for a required argument, negative size,
  * H % G != 0, bad chunk or dtype, misaligned pointer), SSD_ERR_UNSUPPORTED (P, N),
  * SSD_ERR_WORKSPACE (workspace too small or NULL while required), SSD_ERR_CUDA.
@@ -102,6 +104,12 @@ SSD_API int ssd_prefill(int b, int T, int H, int P, int N, int G, int chunk, int
                 const void* x, const float* dt, const float* A, const void* B,
                 const void* C, const float* D, const float* h0, void* y, float* h_final,
                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream` and returns the device-side status recorded by the most recent
+ * ssd_prefill that used `workspace` (SSD_OK, or SSD_ERR_TIMEOUT if a bounded wait inside
+ * the tensor-core kernel expired, or SSD_ERR_INTERNAL for a failed device consistency
+ * check), then clears it.  Each ssd_prefill call resets the status word first. */
+SSD_API int ssd_prefill_check(void* workspace, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * Cached decode step  ([CF-SSD] O(1) caching section)

@@ -21,6 +21,7 @@ from .ssd import (  # noqa: F401
     profile_begin,
     profile_end,
     prefill,
+    prefill_check,
     prefill_workspace_size,
     status_string,
 )

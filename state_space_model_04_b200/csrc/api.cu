@@ -20,6 +20,12 @@ int launch_prefill_simt(int b, int T, int H, int N, int G, int L, int io, const 
                         const float* dt, const float* A, const void* Bm, const void* Cm,
                         const float* D, const float* h0, void* y, float* hf, void* ws,
                         cudaStream_t s);
+bool prefill_tc_supported(int P, int N, int io);
+size_t prefill_tc_workspace_bytes();
+int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt, const float* A, const void* Bm,
+                      const void* Cm, const float* D, const float* h0, void* y, float* hf, void* ws,
+                      cudaStream_t s);
+int prefill_tc_status(void* ws, cudaStream_t s);
 size_t decode_workspace_bytes(int layers, int b, int G);
 int launch_decode_step(int layers, int b, int H, int N, int G, int act, int io, float* h,
                        float* conv_state, const void* xbc, const float* dt, const float* A,
@@ -184,10 +190,24 @@ int ssd_profile_end(ssd_kernel_time* out, int max_entries) {
     return n;
 }
 
+// Prefill workspace: [0, 256) device status word, then the path's scratch.
+static constexpr size_t kStatusBytes = 256;
+
+static size_t prefill_ws_bytes(int b, int T, int H, int P, int N, int chunk, int io) {
+    if (prefill_tc_supported(P, N, io)) return kStatusBytes + prefill_tc_workspace_bytes();
+    return kStatusBytes + prefill_simt_workspace_bytes(b, T, H, N, chunk, io);
+}
+
 size_t ssd_prefill_workspace_size(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype) {
     if (check_prefill_shape(b, T, H, P, N, G, chunk, io_dtype) != SSD_OK) return 0;
     if (b == 0 || T == 0) return 0;
-    return prefill_simt_workspace_bytes(b, T, H, N, chunk, io_dtype);
+    return prefill_ws_bytes(b, T, H, P, N, chunk, io_dtype);
+}
+
+int ssd_prefill_check(void* workspace, void* stream) {
+    g_detail[0] = 0;
+    if (!workspace) return set_error(SSD_ERR_INVALID_ARG, "workspace is NULL");
+    return prefill_tc_status(workspace, static_cast<cudaStream_t>(stream));
 }
 
 int ssd_prefill(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype,
@@ -229,12 +249,18 @@ int ssd_prefill(int b, int T, int H, int P, int N, int G, int chunk, int io_dtyp
             return set_error(SSD_ERR_INVALID_ARG, "h_final overlaps input %s", names[i]);
     }
     if (overlaps(ry, {h_final, h_final ? state_bytes : 0})) return set_error(SSD_ERR_INVALID_ARG, "y overlaps h_final");
-    const size_t need = prefill_simt_workspace_bytes(b, T, H, N, chunk, io_dtype);
-    if (need && (!workspace || workspace_bytes < need))
+    const size_t need = prefill_ws_bytes(b, T, H, P, N, chunk, io_dtype);
+    if (!workspace || workspace_bytes < need)
         return set_error(SSD_ERR_WORKSPACE, "workspace %zu bytes at %p, need %zu", workspace_bytes, workspace, need);
-    if (workspace && !aligned16(workspace)) return set_error(SSD_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    if (!aligned16(workspace)) return set_error(SSD_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    if (overlaps({workspace, need}, ry)) return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps y");
+    for (int i = 0; i < 7; ++i)
+        if (overlaps({workspace, need}, rin[i])) return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps %s", names[i]);
+    if (prefill_tc_supported(P, N, io_dtype))
+        return launch_prefill_tc(b, T, H, G, x, dt, A, B, C, D, h0, y, h_final, workspace, s);
+    SSD_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(int), s));
     return launch_prefill_simt(b, T, H, N, G, chunk, io_dtype, x, dt, A, B, C, D, h0, y, h_final,
-                               workspace, s);
+                               static_cast<char*>(workspace) + kStatusBytes, s);
 }
 
 size_t ssd_decode_workspace_size(int layers, int b, int G) {

@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill_workspace_size.restype = _sz
         L.ssd_prefill.argtypes = [_i] * 8 + [_vp] * 10 + [_sz, _vp]
         L.ssd_prefill.restype = _i
+        L.ssd_prefill_check.argtypes = [_vp, _vp]
+        L.ssd_prefill_check.restype = _i
         L.ssd_decode_workspace_size.argtypes = [_i] * 3
         L.ssd_decode_workspace_size.restype = _sz
         L.ssd_decode_step.argtypes = [_i] * 9 + [_vp] * 10 + [_sz, _vp]
@@ -142,9 +144,10 @@ def prefill_workspace_size(b, T, H, P, N, G, chunk, io_dtype) -> int:
 
 
 def prefill(x, dt, A, B, C, D, chunk=256, h0=None, y=None, h_final=None, workspace=None,
-            want_final=True, stream=None):
+            want_final=True, stream=None, check=False):
     """Chunked SSD prefill.  Shapes: x [b,T,H,P], dt [b,T,H] f32, A [H] f32,
-    B/C [b,T,G,N], D [H] f32, h0 [b,H,P,N] f32 or None.  Returns (y, h_final)."""
+    B/C [b,T,G,N], D [H] f32, h0 [b,H,P,N] f32 or None.  Returns (y, h_final).
+    check=True synchronises and raises if a device-side wait recorded an error."""
     _need(x, "x")
     io = _io(x)
     b, T, H, P = x.shape
@@ -171,7 +174,14 @@ def prefill(x, dt, A, B, C, D, chunk=256, h0=None, y=None, h_final=None, workspa
                            _ptr(C), _ptr(D), _ptr(h0), _ptr(y), _ptr(h_final), _ptr(workspace),
                            ws_bytes, _stream(stream))
     _check(st, "ssd_prefill")
+    if check and workspace is not None:
+        prefill_check(workspace, stream)
     return y, h_final
+
+
+def prefill_check(workspace, stream=None):
+    """Synchronise and raise if the last prefill on `workspace` recorded a device-side error."""
+    _check(lib().ssd_prefill_check(_ptr(workspace), _stream(stream)), "ssd_prefill_check")
 
 
 def decode_workspace_size(layers, b, G) -> int:

@@ -77,6 +77,7 @@ def oracle_subset(case, seqs, heads, nthreads=0):
 
 def run_prefill(ssd, case, chunk=None, **kw):
     t = prefill_inputs(case)
+    kw.setdefault("check", True)
     y, hf = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=chunk or case.L,
                         h0=t["h0"], **kw)
     torch.cuda.synchronize()

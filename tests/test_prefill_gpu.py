@@ -83,6 +83,21 @@ def test_long_context_sampled(L):
     assert torch.isfinite(y.float()).all()
 
 
+def test_fused_kernel_is_the_bf16_path():
+    """bf16 with P=64, N=128 runs the single fused tensor-core kernel; other shapes and fp32
+    run the four-kernel path."""
+    case = make_prefill(1, 512, 4, 64, 128, 1, 256, "bf16", seed=15)
+    ssd.profile_begin()
+    run_prefill(ssd, case)
+    kt = ssd.profile_end()
+    assert list(kt) == ["ssd_prefill_fused"] and kt["ssd_prefill_fused"][0] == 1
+    case = make_prefill(1, 512, 4, 64, 64, 1, 256, "bf16", seed=15)
+    ssd.profile_begin()
+    run_prefill(ssd, case)
+    kt = ssd.profile_end()
+    assert "simt_chunk_output" in kt and "ssd_prefill_fused" not in kt
+
+
 # ------------------------------------------------------------------ invariants
 def test_deterministic_bitwise():
     case = make_prefill(2, 700, 4, 64, 128, 2, 256, "bf16", h0_std=0.1, seed=5)
