@@ -16,20 +16,20 @@
 // as two such blocks with the state handed between them -- the same dual form over a
 // shorter segment, identical in exact arithmetic.
 //
-//   warp 0       TMA producer: C, B (two 64-column 128B-swizzled boxes each) and X per
-//                block into two stages
-//   warp 1       TMEM owner and MMA issuer (one lane), per block t:
-//                  CB(t+1) = C B^T        (M=128 i, N=128 j, K=128 n)   SS   -> TMEM
-//                  S(t)^T  = B^T (w o X)  (M=128 n, N=64 p,  K=128 j)   SS   -> TMEM
-//                  Y(t)    = P X          (M=128 i, N=64 p,  K=128 j)   TS (P in TMEM)
-//                  Yst(t)  = C H^T        (M=128 i, N=64 p,  K=128 n)   SS
-//   warps 2-9    "scores" group (2 warps per TMEM lane quadrant): prefix sum of dt*A,
-//                w o X into shared memory, and the decayed causal scores P = bf16(CB o L)
-//                written back into TMEM as the A operand of the next MMA
-//   warps 10-17  "state" group (2 warps per quadrant): H <- exp(cs_last) H + S (fp32,
-//                registers), bf16 H^T for the next C H^T, y = Y + exp(cs_i) Yst, TMA store
-// The scores group runs one block ahead of the state group, so the tensor core, the TMA
-// engine and both epilogues overlap.
+//   warp 0       TMA producer: C and B (two 64-column 128B-swizzled boxes each) into a
+//                2-slot ring, X into a 3-slot ring
+//   warp 1       TMEM owner and MMA issuer (one lane).  Iteration k:
+//                  Y(k)      = P(k) X(k)      (M=128 i, N=64 p,  K=128 j)  TS, P in TMEM
+//                  CB(k+1)   = C B^T          (M=128 i, N=128 j, K=128 n)  SS
+//                  Yst(k+1)  = C H^T          (M=128 i, N=64 p,  K=128 n)  SS
+//                  S(k+1)^T  = B^T (w o X)    (M=128 n, N=64 p,  K=128 j)  SS
+//                so C and B of a block are dead within one iteration and the next
+//                block's loads run a full iteration ahead of their use.
+//   warps 2-9    "scores" group (2 warps per TMEM lane quadrant): prefix sum of dt*A and
+//                P = bf16(CB o L), written back into TMEM as the A operand of P X
+//   warps 10-17  "state" group (2 warps per quadrant): prefix sums, w o X into shared
+//                memory, H <- exp(cs_last) H + S (fp32 registers) with its bf16 copy for
+//                C H^T, and y = Y + exp(cs_i) Yst stored straight from registers
 //
 // Decay arithmetic.  Below the 32x32 diagonal sub-blocks the decay factorises exactly
 // as exp(cs_i - cs_e) * exp(cs_e - cs_j) with e the last token of j's 32-token group
@@ -57,44 +57,58 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t kRegion = kBlk * 128;             // one [128 rows][64 bf16] swizzled box: 16 KB
-constexpr uint32_t kStageC = 0;                      // 2 regions (n 0..63, 64..127)
-constexpr uint32_t kStageB = 2 * kRegion;            // 2 regions
-constexpr uint32_t kStageX = 4 * kRegion;            // 1 region
-constexpr uint32_t kStageBytes = 5 * kRegion;        // 80 KB
-constexpr uint32_t kXs = 2 * kStageBytes;            // two w o X buffers
-constexpr uint32_t kSH = kXs + 2 * kRegion;          // bf16 H^T [n][p]
-constexpr uint32_t kYst = kSH + kRegion;             // y staging tile for the TMA store
-constexpr uint32_t kSmall = kYst + kRegion;          // barriers and per-token scalars
-constexpr uint32_t kSmallBytes = 2560;
+constexpr uint32_t kCBSlot = 4 * kRegion;            // C (2 regions: n 0..63, 64..127) then B (2)
+constexpr uint32_t kSlotC = 0;
+constexpr uint32_t kSlotB = 2 * kRegion;
+constexpr uint32_t kXRing = 2 * kCBSlot;             // 3 X slots of one region
+constexpr uint32_t kXs = kXRing + 3 * kRegion;       // w o X
+constexpr uint32_t kSH = kXs + kRegion;              // bf16 H^T [n][p]
+constexpr uint32_t kSmall = kSH + kRegion;           // barriers and per-token scalars
+constexpr uint32_t kSmallBytes = 4096;
 constexpr uint32_t kSmemBytes = kSmall + kSmallBytes;
-constexpr uint32_t kTxBytes = 5 * kRegion;           // bytes landing per stage
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // TMEM columns (512 x 128 lanes x 32 bit)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColCB = 0;      // two 128-column fp32 C B^T buffers; S(t) reuses buffer t%2
-constexpr uint32_t kColP = 256;     // bf16 scores, 2 per column (64 columns)
-constexpr uint32_t kColY = 320;     // two 64-column Y buffers
-constexpr uint32_t kColYst = 448;   // 64 columns
+constexpr uint32_t kColCB = 0;      // fp32 C B^T (128 columns)
+constexpr uint32_t kColP = 128;     // bf16 scores, 2 per column (64 columns)
+constexpr uint32_t kColS = 192;     // fp32 S^T (64 columns)
+constexpr uint32_t kColY = 256;     // two 64-column Y buffers
+constexpr uint32_t kColYst = 384;   // two 64-column C H^T buffers
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 // barrier indices in the small area
 enum {
-    BAR_FULL0 = 0, BAR_FULL1, BAR_EMPTY0, BAR_EMPTY1, BAR_CB0, BAR_CB1, BAR_ACCS0, BAR_ACCS1,
-    BAR_SCORES, BAR_PFREE, BAR_SFREE, BAR_ACCY, BAR_H, BAR_DONE, BAR_COUNT
+    BAR_FULLCB = 0,   // [2] C,B landed
+    BAR_EMPTYCB = 2,  // [2] C,B slot released by the MMAs
+    BAR_FULLX = 4,    // [3] X landed
+    BAR_EMPTYX = 7,   // [3] X slot released
+    BAR_CBFULL = 10,  // C B^T accumulated
+    BAR_CBFREE,       // scores group has read C B^T            (256 arrivals)
+    BAR_XS,           // state group has written w o X          (256)
+    BAR_ACCS,         // S^T accumulated (and w o X read)
+    BAR_SFREE,        // state group has read S^T               (256)
+    BAR_YSTDONE,      // C H^T accumulated (and bf16 H read)
+    BAR_H,            // state group has written bf16 H         (256)
+    BAR_SCORES,       // scores group has written P             (256)
+    BAR_G2DONE,       // P X accumulated (and P read)
+    BAR_YFREE0,       // [2] scores group has read Y and C H^T of the slot (256)
+    BAR_PREP0 = BAR_YFREE0 + 2,  // [2] state group has published a block's decay arrays (256)
+    BAR_DONE = BAR_PREP0 + 2,
+    BAR_COUNT
 };
 
 struct TcParams {
     CUtensorMap tm_x;
     CUtensorMap tm_B;
     CUtensorMap tm_C;
-    CUtensorMap tm_y;
     const float* dt;
     const float* A;
     const float* D;
     const float* h0;
     float* hf;
+    __nv_bfloat16* y;
     int* status;
     int T, H, G, nblk;
 };
@@ -128,6 +142,19 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait that lets the hardware suspend the thread (up to ~1 ms) until the phase
+// completes, instead of spinning on the issue slots other warps need.
+__device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(1000000u)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait for the phase with `parity` to complete.  Returns false (and makes every
 // other role give up) if the CTA is aborting or the limit expires.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -135,7 +162,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
-        if (mbar_try(bar, parity)) return true;
+        if (mbar_try_sleep(bar, parity)) return true;
         if (*abort_flag) return false;
         if (globaltimer() - t0 > kWaitLimitNs) {
             *abort_flag = 1;
@@ -164,14 +191,6 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm,
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap* tm, uint32_t src, int c0, int c1, int c2, int c3) {
-    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
-                 ::"l"(reinterpret_cast<uint64_t>(tm)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -199,27 +218,33 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, 
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-__device__ __forceinline__ void mma_ss(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// Whole-warp variants: every lane runs the issuing code (so its operands stay warp-uniform)
+// and one elected lane executes the instruction.
+__device__ __forceinline__ void mma_ss_w(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
         ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
-__device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc, uint32_t acc) {
+__device__ __forceinline__ void mma_ts_w(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
         ::"r"(tmem_d), "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
+__device__ __forceinline__ void mma_commit_w(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(bar)
+        : "memory");
 }
-
 #define SSD_TMEM_LD32(taddr, r)                                                                          \
     asm volatile(                                                                                        \
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15," \
@@ -295,13 +320,14 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 
     uint8_t* small = smem + kSmall;
     uint64_t* bars = reinterpret_cast<uint64_t*>(small);              // BAR_COUNT barriers
-    float* s_m = reinterpret_cast<float*>(small + 128);               // [2][128] log2(dt_j) - cs_j log2e
+    // per-token decay arrays of a block, published by the state group for the scores group
+    float* s_m = reinterpret_cast<float*>(small + 256);               // [2][128] log2(dt_j) - cs_j log2e
     float* s_v = s_m + 2 * kBlk;                                      // [2][128] exp(cs_e - cs_j) dt_j
-    float* s_stot = s_v + 2 * kBlk;                                   // [2][4] scores-group quadrant sums
-    float* s_ytot = s_stot + 8;                                       // [2][4] state-group quadrant sums
+    float* s_cs = s_v + 2 * kBlk;                                     // [2][128] cs_i
+    float* s_cend = s_cs + 2 * kBlk;                                  // [2][4] cs at the end of each 32-token group
+    float* s_ytot = s_cend + 8;                                       // [2][4] state-group quadrant sums
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_ytot + 8);
-    volatile int* s_sstop = s_abort + 1;                              // [2]
-    volatile int* s_ystop = s_abort + 3;                              // [2]
+    volatile int* s_ystop = s_abort + 1;                              // [2]
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_ytot + 16);
 
     const uint32_t sbase = smem_u32(smem);
@@ -310,22 +336,13 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     if (threadIdx.x == 0) {
         const bool misaligned = (sbase & 1023u) != 0;  // swizzled layouts need a 1024-byte base
         if (misaligned) atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (1 << 8));
-        mbar_init(bar(BAR_FULL0), 1);
-        mbar_init(bar(BAR_FULL1), 1);
-        mbar_init(bar(BAR_EMPTY0), 1);
-        mbar_init(bar(BAR_EMPTY1), 1);
-        mbar_init(bar(BAR_CB0), 1);
-        mbar_init(bar(BAR_CB1), 1);
-        mbar_init(bar(BAR_ACCS0), 1);
-        mbar_init(bar(BAR_ACCS1), 1);
-        mbar_init(bar(BAR_SCORES), kGroupThreads);
-        mbar_init(bar(BAR_PFREE), 1);
-        mbar_init(bar(BAR_SFREE), kGroupThreads);
-        mbar_init(bar(BAR_ACCY), 1);
-        mbar_init(bar(BAR_H), kGroupThreads);
-        mbar_init(bar(BAR_DONE), 1);
+        for (int i = 0; i < BAR_COUNT; ++i) {
+            const bool group = (i == BAR_CBFREE || i == BAR_XS || i == BAR_SFREE || i == BAR_H ||
+                                i == BAR_SCORES || i == BAR_YFREE0 || i == BAR_YFREE0 + 1 || i == BAR_PREP0 ||
+                                i == BAR_PREP0 + 1);
+            mbar_init(bar(i), group ? kGroupThreads : 1);
+        }
         *s_abort = misaligned ? 1 : 0;
-        s_sstop[0] = s_sstop[1] = 0;
         s_ystop[0] = s_ystop[1] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -343,83 +360,117 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         // ================================================================ TMA producer
         if (lane == 0 && !*s_abort) {
             int issued = 0;
-            for (int t = 0; t < nblk; ++t) {
-                const int s = t & 1;
-                if (t >= 2 && !mbar_wait(bar(BAR_EMPTY0 + s), ((t - 2) >> 1) & 1, s_abort, prm.status, 1)) break;
-                const uint32_t full = bar(BAR_FULL0 + s);
-                const uint32_t st = sbase + s * kStageBytes;
-                mbar_expect_tx(full, kTxBytes);
-                const int t0 = t * kBlk;
-                tma_load_4d(st + kStageC, &prm.tm_C, full, 0, g, t0, bi);
-                tma_load_4d(st + kStageC + kRegion, &prm.tm_C, full, 64, g, t0, bi);
-                tma_load_4d(st + kStageB, &prm.tm_B, full, 0, g, t0, bi);
-                tma_load_4d(st + kStageB + kRegion, &prm.tm_B, full, 64, g, t0, bi);
-                tma_load_4d(st + kStageX, &prm.tm_x, full, 0, hd, t0, bi);
-                issued = t + 1;
+            for (int u = 0; u < nblk; ++u) {
+                const int s2 = u & 1, s3 = u % 3;
+                const int t0 = u * kBlk;
+                if (u >= 2 && !mbar_wait(bar(BAR_EMPTYCB + s2), ((u - 2) >> 1) & 1, s_abort, prm.status, 1)) break;
+                const uint32_t fcb = bar(BAR_FULLCB + s2);
+                const uint32_t slot = sbase + s2 * kCBSlot;
+                mbar_expect_tx(fcb, 4 * kRegion);
+                tma_load_4d(slot + kSlotC, &prm.tm_C, fcb, 0, g, t0, bi);
+                tma_load_4d(slot + kSlotC + kRegion, &prm.tm_C, fcb, 64, g, t0, bi);
+                tma_load_4d(slot + kSlotB, &prm.tm_B, fcb, 0, g, t0, bi);
+                tma_load_4d(slot + kSlotB + kRegion, &prm.tm_B, fcb, 64, g, t0, bi);
+                if (u >= 3 && !mbar_wait(bar(BAR_EMPTYX + s3), ((u - 3) / 3) & 1, s_abort, prm.status, 2)) {
+                    issued = -(u + 1);  // C,B of block u issued, X not
+                    break;
+                }
+                const uint32_t fx = bar(BAR_FULLX + s3);
+                mbar_expect_tx(fx, kRegion);
+                tma_load_4d(sbase + kXRing + s3 * kRegion, &prm.tm_x, fx, 0, hd, t0, bi);
+                issued = u + 1;
             }
-            // the last (up to) two stages may hold loads nobody waited for: let them land
-            for (int u = issued - 2; u < issued; ++u)
-                if (u >= 0) mbar_drain(bar(BAR_FULL0 + (u & 1)), (u >> 1) & 1);
+            // loads nobody may have waited for must land before the CTA exits
+            const int ncb = issued < 0 ? -issued : issued;  // blocks whose C,B were issued
+            const int nx = issued < 0 ? -issued - 1 : issued;
+            for (int u = ncb - 2; u < ncb; ++u)
+                if (u >= 0) mbar_drain(bar(BAR_FULLCB + (u & 1)), (u >> 1) & 1);
+            for (int u = nx - 3; u < nx; ++u)
+                if (u >= 0) mbar_drain(bar(BAR_FULLX + u % 3), (u / 3) & 1);
         }
     } else if (warp == 1) {
         // ================================================================ MMA issuer
-        if (lane == 0 && !*s_abort) {
-            constexpr uint32_t id_cb = idesc_bf16(128, 128, 0, 0);   // A C (K-major), B B (K-major)
-            constexpr uint32_t id_s = idesc_bf16(128, 64, 1, 1);     // A B^T (MN-major), B w o X (MN-major)
-            constexpr uint32_t id_y = idesc_bf16(128, 64, 0, 1);     // A P (TMEM), B X (MN-major)
-            constexpr uint32_t id_yst = idesc_bf16(128, 64, 0, 1);   // A C (K-major), B H^T (MN-major)
-            auto issue_cb = [&](int u) {
-                const uint32_t st = sbase + (u & 1) * kStageBytes;
-                const uint32_t d = tmem + kColCB + (u & 1) * 128;
+        // The whole warp runs this loop (operands stay warp-uniform); one elected lane
+        // issues each tcgen05 instruction.
+        constexpr uint32_t id_cb = idesc_bf16(128, 128, 0, 0);   // A C (K-major), B B (K-major)
+        constexpr uint32_t id_s = idesc_bf16(128, 64, 1, 1);     // A B^T (MN-major), B w o X (MN-major)
+        constexpr uint32_t id_y = idesc_bf16(128, 64, 0, 1);     // A P (TMEM), B X (MN-major)
+        constexpr uint32_t id_yst = idesc_bf16(128, 64, 0, 1);   // A C (K-major), B H^T (MN-major)
+        auto wt = [&](int b, uint32_t parity, int where) {
+            return warp_wait(bar(b), parity, s_abort, prm.status, where);
+        };
+        auto issue_cb = [&](int u) {  // C B^T of block u (C, B in ring slot u & 1)
+            const uint32_t slot = sbase + (u & 1) * kCBSlot;
+            const uint64_t dC = sdesc(slot + kSlotC, 16, 1024), dB = sdesc(slot + kSlotB, 16, 1024);
+            // a K step of 16 advances only the 16-byte address field of a K-major descriptor
 #pragma unroll
-                for (int k = 0; k < kN / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kRegion + (k & 3) * 32;
-                    mma_ss(d, sdesc(st + kStageC + off, 16, 1024), sdesc(st + kStageB + off, 16, 1024), id_cb, k > 0);
-                }
-                mma_commit(bar(BAR_CB0 + (u & 1)));
-            };
-            bool ok = mbar_wait(bar(BAR_FULL0), 0, s_abort, prm.status, 2);
-            if (ok) {
-                tc_fence_after();
-                issue_cb(0);
+            for (int k = 0; k < kN / 16; ++k) {
+                const uint32_t off = (k >> 2) * (kRegion >> 4) + (k & 3) * 2;
+                mma_ss_w(tmem + kColCB, dC + off, dB + off, id_cb, k > 0);
             }
-            for (int t = 0; t < nblk && ok; ++t) {
-                const int s = t & 1;
-                const uint32_t st = sbase + s * kStageBytes;
-                // (a) C B^T of the next block, into the buffer whose S was consumed
-                if (t + 1 < nblk) {
-                    if (!(ok = mbar_wait(bar(BAR_FULL0 + (s ^ 1)), ((t + 1) >> 1) & 1, s_abort, prm.status, 3))) break;
-                    if (t >= 1 && !(ok = mbar_wait(bar(BAR_SFREE), (t - 1) & 1, s_abort, prm.status, 4))) break;
+            mma_commit_w(bar(BAR_CBFULL));
+        };
+        auto issue_yst = [&](int u) {  // C H_u^T
+            const uint32_t slot = sbase + (u & 1) * kCBSlot;
+            const uint64_t dC = sdesc(slot + kSlotC, 16, 1024), dH = sdesc(sbase + kSH, kRegion, 1024);
+#pragma unroll
+            for (int k = 0; k < kN / 16; ++k) {
+                const uint32_t off = (k >> 2) * (kRegion >> 4) + (k & 3) * 2;
+                mma_ss_w(tmem + kColYst + (u & 1) * 64, dC + off, dH + k * 128, id_yst, k > 0);  // MN step: 16 rows
+            }
+            mma_commit_w(bar(BAR_YSTDONE));
+        };
+        auto issue_state = [&](int u) {  // S_u^T = B^T (w o X); then C, B of block u are dead
+            const uint32_t slot = sbase + (u & 1) * kCBSlot;
+            const uint64_t dBt = sdesc(slot + kSlotB, kRegion, 1024), dXs = sdesc(sbase + kXs, kRegion, 1024);
+#pragma unroll
+            for (int k = 0; k < kBlk / 16; ++k) mma_ss_w(tmem + kColS, dBt + k * 128, dXs + k * 128, id_s, k > 0);
+            mma_commit_w(bar(BAR_ACCS));
+            mma_commit_w(bar(BAR_EMPTYCB + (u & 1)));
+        };
+        auto issue_y = [&](int k) {  // Y_k = P_k X_k; then X of block k is dead
+            const uint64_t dX = sdesc(sbase + kXRing + (k % 3) * kRegion, kRegion, 1024);
+#pragma unroll
+            for (int kk = 0; kk < kBlk / 16; ++kk)
+                mma_ts_w(tmem + kColY + (k & 1) * 64, tmem + kColP + kk * 8, dX + kk * 128, id_y, kk > 0);
+            mma_commit_w(bar(BAR_G2DONE));
+            mma_commit_w(bar(BAR_EMPTYX + k % 3));
+        };
+        bool ok = __all_sync(0xffffffffu, !*s_abort);
+        if (ok) {
+            // block 0: C B^T, C H_0^T, S_0
+            ok = wt(BAR_FULLCB, 0, 3);
+            if (ok) { tc_fence_after(); issue_cb(0); ok = wt(BAR_H, 0, 5); }
+            if (ok) { tc_fence_after(); issue_yst(0); ok = wt(BAR_XS, 0, 6); }
+            if (ok) { tc_fence_after(); issue_state(0); }
+            // iteration k: C B^T(k+1) first (the scores group's longest lead), then P X (k),
+            // C H^T (k+1) and S(k+1)
+            for (int k = 0; k < nblk && ok; ++k) {
+                if (k + 1 < nblk) {
+                    ok = wt(BAR_FULLCB + ((k + 1) & 1), ((k + 1) >> 1) & 1, 7) && wt(BAR_CBFREE, k & 1, 4);
+                    if (!ok) break;
                     tc_fence_after();
-                    issue_cb(t + 1);
+                    issue_cb(k + 1);
                 }
-                // (b) S(t)^T = B^T (w o X) into buffer s; Y(t) = P X
-                if (!(ok = mbar_wait(bar(BAR_SCORES), t & 1, s_abort, prm.status, 5))) break;
+                // Y and C H^T buffers k & 1 were last read for block k - 2
+                ok = wt(BAR_FULLX + k % 3, (k / 3) & 1, 8) && wt(BAR_SCORES, k & 1, 9) &&
+                     (k < 2 || wt(BAR_YFREE0 + (k & 1), ((k - 2) >> 1) & 1, 10));
+                if (!ok) break;
                 tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < kBlk / 16; ++k)
-                    mma_ss(tmem + kColCB + s * 128, sdesc(st + kStageB + k * 2048, kRegion, 1024),
-                           sdesc(sbase + kXs + s * kRegion + k * 2048, kRegion, 1024), id_s, k > 0);
-                mma_commit(bar(BAR_ACCS0 + s));
-#pragma unroll
-                for (int k = 0; k < kBlk / 16; ++k)
-                    mma_ts(tmem + kColY + s * 64, tmem + kColP + k * 8, sdesc(st + kStageX + k * 2048, kRegion, 1024),
-                           id_y, k > 0);
-                mma_commit(bar(BAR_PFREE));
-                // (c) Yst(t) = C H_t^T
-                if (!(ok = mbar_wait(bar(BAR_H), t & 1, s_abort, prm.status, 6))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < kN / 16; ++k) {
-                    const uint32_t offa = (k >> 2) * kRegion + (k & 3) * 32;
-                    mma_ss(tmem + kColYst, sdesc(st + kStageC + offa, 16, 1024),
-                           sdesc(sbase + kSH + k * 2048, kRegion, 1024), id_yst, k > 0);
+                issue_y(k);
+                if (k + 1 < nblk) {
+                    ok = wt(BAR_H, (k + 1) & 1, 5);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_yst(k + 1);
+                    ok = wt(BAR_XS, (k + 1) & 1, 6) && wt(BAR_SFREE, k & 1, 11);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_state(k + 1);
                 }
-                mma_commit(bar(BAR_ACCY));
-                mma_commit(bar(BAR_EMPTY0 + s));
             }
             // every MMA and commit issued above completes before the TMEM is released
-            mma_commit(bar(BAR_DONE));
+            mma_commit_w(bar(BAR_DONE));
             mbar_drain(bar(BAR_DONE), 0);
         }
     } else if (warp < 10) {
@@ -427,74 +478,82 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         const int q = warp & 3, half = (warp - 2) >> 2;
         const int r = q * 32 + lane;  // token row i (and column index j for the per-token arrays)
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-        const float Ah = prm.A[hd], Dh = prm.D[hd];
+        const float Dh = prm.D[hd];
+        const int p0 = half * 32;  // this warp's 32 of the 64 p columns of the output
+        // y(k) = Y(k) + exp(cs_i) Yst(k) for row r, columns [p0, p0 + 32), straight to global.
+        // exp(cs_i) is carried in a register: by now the state group may have republished
+        // the per-token arrays of block k's slot.
+        auto store_y = [&](int k, float ei) {
+            tc_fence_after();
+            uint32_t yp[16];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t ry[16], rs[16];
+                SSD_TMEM_LD16(tmem + lane_addr + kColY + (k & 1) * 64 + p0 + hh * 16, ry);
+                SSD_TMEM_LD16(tmem + lane_addr + kColYst + (k & 1) * 64 + p0 + hh * 16, rs);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    yp[hh * 8 + j] = pack_bf16(fmaf(ei, __uint_as_float(rs[2 * j]), __uint_as_float(ry[2 * j])),
+                                               fmaf(ei, __uint_as_float(rs[2 * j + 1]), __uint_as_float(ry[2 * j + 1])));
+            }
+            tc_fence_before();
+            mbar_arrive(bar(BAR_YFREE0 + (k & 1)));
+            const int tok = k * kBlk + r;
+            if (tok < T) {
+                uint4* dst = reinterpret_cast<uint4*>(prm.y + (((size_t)bi * T + tok) * H + hd) * kP + p0);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)
+                    dst[c4] = make_uint4(yp[4 * c4], yp[4 * c4 + 1], yp[4 * c4 + 2], yp[4 * c4 + 3]);
+            }
+        };
         bool live = __all_sync(0xffffffffu, !*s_abort);
-        for (int t = 0; t < nblk; ++t) {
-            const int s = t & 1;
-            const int t0 = t * kBlk;
-            // ---- prefix sums; per-token arrays for block t (slot s)
-            const float dtv = (t0 + r < T) ? prm.dt[((size_t)bi * T + t0 + r) * H + hd] : 0.f;
-            if (!live || *s_abort) s_sstop[s] = 1;
-            float cend[4], cs_last;
-            const float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_stot + s * 4, 2, cs_last, cend);
-            if (s_sstop[s]) break;  // identical for the whole group (read after its barrier)
-            if (half == 0) {
-                s_m[s * kBlk + r] = __log2f(dtv) - cs * kLog2e;                 // -inf where dt = 0
-                s_v[s * kBlk + r] = __expf(cend[q] - cs) * dtv;                  // cend[q]: end of j's quadrant
-            }
-            group_bar(2);
-            const float w = __expf(cs_last - cs) * dtv;
-
-            // ---- w o X into Xs[s] (row r = token j; this warp's 4 of the 8 chunks)
-            if (live) live = warp_wait(bar(BAR_FULL0 + s), (t >> 1) & 1, s_abort, prm.status, 7);
-            if (live && t >= 2) live = warp_wait(bar(BAR_ACCS0 + s), ((t - 2) >> 1) & 1, s_abort, prm.status, 8);
-            if (live) {
-                const uint8_t* src = smem + s * kStageBytes + kStageX;
-                uint8_t* dst = smem + kXs + s * kRegion;
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const int c = half * 4 + c4;
-                    uint4 u = *reinterpret_cast<const uint4*>(src + swz(r, c));
-                    uint32_t* e = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&e[k]));
-                        e[k] = pack_bf16(f.x * w, f.y * w);
-                    }
-                    *reinterpret_cast<uint4*>(dst + swz(r, c)) = u;
-                }
-            }
+        float ei_prev = 0.f;  // exp(cs_i) of the previous block
+        for (int u = 0; u < nblk; ++u) {
+            const int s = u & 1;
+            float ei_cur = 0.f;
+            // the state group publishes cs, the chunk ends and the per-column decay terms
+            if (live) live = warp_wait(bar(BAR_PREP0 + s), (u >> 1) & 1, s_abort, prm.status, 17);
             // ---- P = bf16(CB o L) for this warp's chunks {half, half + 2} of row r
-            if (live) live = warp_wait(bar(BAR_CB0 + s), (t >> 1) & 1, s_abort, prm.status, 9);
+            uint32_t pk[2][16];
+            if (live) live = warp_wait(bar(BAR_CBFULL), u & 1, s_abort, prm.status, 11);
             if (live) {
                 tc_fence_after();
                 const float* vs = s_v + s * kBlk;
                 const float* ms = s_m + s * kBlk;
+                const float cs = s_cs[s * kBlk + r];
                 const float csl = cs * kLog2e;
-                bool pfree_seen = (t == 0);
+                ei_cur = __expf(cs);
+                float cend[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) cend[c] = s_cend[s * 4 + c];
+                // chunk by chunk; C B^T is released as soon as the last chunk has been read
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c = half + 2 * cc;
-                    uint32_t pk[16];
-                    if (c < q) {  // below the diagonal sub-block: factorised decay
-                        uint32_t raw[32];
-                        SSD_TMEM_LD32(tmem + lane_addr + kColCB + s * 128 + c * 32, raw);
-                        const float u = __expf(cs - cend[c]);
+                    uint32_t raw[32];
+                    if (c <= q) {
+                        SSD_TMEM_LD32(tmem + lane_addr + kColCB + c * 32, raw);
                         tmem_wait_ld();
+                    }
+                    if (cc == 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(BAR_CBFREE));
+                    }
+                    if (c < q) {  // below the diagonal sub-block: factorised decay
+                        const float ce = (c == 0) ? cend[0] : (c == 1) ? cend[1] : cend[2];
+                        const float uu = __expf(cs - ce);
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
                             const float4 v4 = *reinterpret_cast<const float4*>(vs + c * 32 + 4 * k);
-                            const float a0 = __uint_as_float(raw[4 * k + 0]) * u;
-                            const float a1 = __uint_as_float(raw[4 * k + 1]) * u;
-                            const float a2 = __uint_as_float(raw[4 * k + 2]) * u;
-                            const float a3 = __uint_as_float(raw[4 * k + 3]) * u;
-                            pk[2 * k] = pack_bf16(a0 * v4.x, a1 * v4.y);
-                            pk[2 * k + 1] = pack_bf16(a2 * v4.z, a3 * v4.w);
+                            const float a0 = __uint_as_float(raw[4 * k + 0]) * uu;
+                            const float a1 = __uint_as_float(raw[4 * k + 1]) * uu;
+                            const float a2 = __uint_as_float(raw[4 * k + 2]) * uu;
+                            const float a3 = __uint_as_float(raw[4 * k + 3]) * uu;
+                            pk[cc][2 * k] = pack_bf16(a0 * v4.x, a1 * v4.y);
+                            pk[cc][2 * k + 1] = pack_bf16(a2 * v4.z, a3 * v4.w);
                         }
                     } else if (c == q) {  // diagonal sub-block: per-element decay and causal mask
-                        uint32_t raw[32];
-                        SSD_TMEM_LD32(tmem + lane_addr + kColCB + s * 128 + c * 32, raw);
-                        tmem_wait_ld();
 #pragma unroll
                         for (int k = 0; k < 16; ++k) {
                             const int j0 = 2 * k, j1 = 2 * k + 1;  // column within the sub-block
@@ -503,30 +562,35 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                             float v1 = (j1 <= lane) ? __uint_as_float(raw[j1]) * ex2(csl + m2.y) : 0.f;
                             if (j0 == lane) v0 += Dh;
                             if (j1 == lane) v1 += Dh;
-                            pk[k] = pack_bf16(v0, v1);
+                            pk[cc][k] = pack_bf16(v0, v1);
                         }
                     } else {
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) pk[k] = 0u;
+                        for (int k = 0; k < 16; ++k) pk[cc][k] = 0u;
                     }
-                    if (!pfree_seen) {  // the previous block's P X must be done reading P
-                        live = warp_wait(bar(BAR_PFREE), (t - 1) & 1, s_abort, prm.status, 10);
-                        pfree_seen = true;
-                        if (!live) break;
-                        tc_fence_after();
-                    }
-                    SSD_TMEM_ST16(tmem + lane_addr + kColP + c * 16, pk);
                 }
-                if (live) tmem_wait_st();
+                // the previous block's P X must be done reading P
+                if (u >= 1) live = warp_wait(bar(BAR_G2DONE), (u - 1) & 1, s_abort, prm.status, 12);
+                if (live) {
+                    tc_fence_after();
+                    SSD_TMEM_ST16(tmem + lane_addr + kColP + half * 16, pk[0]);
+                    SSD_TMEM_ST16(tmem + lane_addr + kColP + (half + 2) * 16, pk[1]);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar(BAR_SCORES));
+                }
+                // the previous block's output, once P is published (P X of block u-1 is done)
+                if (live && u >= 1) store_y(u - 1, ei_prev);
             }
-            fence_proxy_async();
-            tc_fence_before();
-            if (live) mbar_arrive(bar(BAR_SCORES));
+            ei_prev = ei_cur;
         }
+        // output of the last block
+        if (live && nblk > 0) live = warp_wait(bar(BAR_G2DONE), (nblk - 1) & 1, s_abort, prm.status, 18);
+        if (live && nblk > 0) store_y(nblk - 1, ei_prev);
     } else {
         // ================================================================ state group
         const int q = warp & 3, half = (warp - 10) >> 2;
-        const int r = q * 32 + lane;  // state row n (state update) and token row i (output)
+        const int r = q * 32 + lane;  // token row (w o X, y) and state row n (S, H)
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
         const float Ah = prm.A[hd];
         const size_t hbase = ((size_t)bi * H + hd) * kP * kN;
@@ -551,79 +615,90 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         mbar_arrive(bar(BAR_H));
         bool live = __all_sync(0xffffffffu, !*s_abort);
         bool stopped = false;
-        const bool leader = (warp == 10 && lane == 0);
-        for (int t = 0; t < nblk; ++t) {
-            const int s = t & 1;
-            const int t0 = t * kBlk;
-            const float dtv = (t0 + r < T) ? prm.dt[((size_t)bi * T + t0 + r) * H + hd] : 0.f;
+        auto load_dt = [&](int u) {
+            const int tok = u * kBlk + r;
+            return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;
+        };
+        // dt is fetched two blocks ahead: under full HBM load its latency is microseconds
+        float dt_a = load_dt(0), dt_b = load_dt(1);
+        float cs_last_prev = 0.f;  // total of the block whose state update is next
+        // iteration k: inputs of block k+1 (w o X), state and output of block k
+        for (int k = -1; k < nblk; ++k) {
+            const int s = (k + 1) & 1;
+            const float dtv = dt_a;
+            dt_a = dt_b;
+            dt_b = load_dt(k + 3);
             if (!live || *s_abort) s_ystop[s] = 1;
             float cend[4], cs_last;
             const float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_ytot + s * 4, 3, cs_last, cend);
             if (s_ystop[s]) { stopped = true; break; }
-            const float gam = __expf(cs_last);
-            const float ei = __expf(cs);
-
-            // ---- H <- exp(cs_last) H + S(t)   (S(t)^T lives in C B^T buffer s)
-            if (live) live = warp_wait(bar(BAR_ACCS0 + s), (t >> 1) & 1, s_abort, prm.status, 11);
-            if (live) {
+            // ---- w o X of block k+1 (needs S^T(k) accumulated: the MMA has read Xs(k))
+            if (live && k >= 0) live = warp_wait(bar(BAR_ACCS), k & 1, s_abort, prm.status, 13);
+            // ---- publish block k+1's decay arrays for the scores group.  S^T(k) being
+            //      accumulated means the scores group is done with block k-1 (same slot).
+            if (live && k + 1 < nblk) {
+                if (half == 0) {
+                    s_cs[s * kBlk + r] = cs;
+                    s_m[s * kBlk + r] = __log2f(dtv) - cs * kLog2e;   // -inf where dt = 0
+                    s_v[s * kBlk + r] = __expf(cend[q] - cs) * dtv;    // cend[q]: end of j's 32-token group
+                    if (r < 4) s_cend[s * 4 + r] = cend[r];
+                }
+                mbar_arrive(bar(BAR_PREP0 + s));
+            }
+            if (k >= 0 && live) {
+                // ---- H <- exp(cs_last(k)) H + S(k)
                 tc_fence_after();
-                uint32_t raw[32];
-                SSD_TMEM_LD32(tmem + lane_addr + kColCB + s * 128 + p0, raw);
-                tmem_wait_ld();
+                {
+                    uint32_t raw[32];
+                    SSD_TMEM_LD32(tmem + lane_addr + kColS + p0, raw);
+                    tmem_wait_ld();
+                    const float gam = __expf(cs_last_prev);
 #pragma unroll
-                for (int k = 0; k < 32; ++k) Hs[k] = fmaf(gam, Hs[k], __uint_as_float(raw[k]));
+                    for (int j = 0; j < 32; ++j) Hs[j] = fmaf(gam, Hs[j], __uint_as_float(raw[j]));
+                }
                 tc_fence_before();
                 mbar_arrive(bar(BAR_SFREE));
-            }
-            // ---- y(t) = Y(t) + exp(cs_i) Yst(t); then hand H_{t+1} to the next C H^T
-            uint32_t yp[16];
-            if (live) live = warp_wait(bar(BAR_ACCY), t & 1, s_abort, prm.status, 12);
-            if (live) {
-                tc_fence_after();
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t ry[16], rs[16];
-                    SSD_TMEM_LD16(tmem + lane_addr + kColY + s * 64 + p0 + hh * 16, ry);
-                    SSD_TMEM_LD16(tmem + lane_addr + kColYst + p0 + hh * 16, rs);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        yp[hh * 8 + k] = pack_bf16(fmaf(ei, __uint_as_float(rs[2 * k]), __uint_as_float(ry[2 * k])),
-                                                   fmaf(ei, __uint_as_float(rs[2 * k + 1]), __uint_as_float(ry[2 * k + 1])));
+                // ---- bf16 H_{k+1} for C H^T of block k+1, once C H^T of block k has read H_k
+                live = warp_wait(bar(BAR_YSTDONE), k & 1, s_abort, prm.status, 15);
+                if (live) {
+                    write_sh();
+                    fence_proxy_async();
+                    mbar_arrive(bar(BAR_H));
                 }
-                write_sh();  // C H_t^T (read by Yst(t)) has completed
-                fence_proxy_async();
-                tc_fence_before();
-                mbar_arrive(bar(BAR_H));
             }
-            // ---- stage y(t) and store it with TMA
-            if (leader) bulk_wait_read0();  // the previous tile has left the staging buffer
-            group_bar(3);
-            if (live) {
-                uint8_t* dst = smem + kYst;
+            // ---- w o X of block k+1 (after the H hand-off: C H^T needs H sooner than the
+            //      state MMA needs w o X)
+            if (live && k + 1 < nblk) {
+                live = warp_wait(bar(BAR_FULLX + (k + 1) % 3), ((k + 1) / 3) & 1, s_abort, prm.status, 14);
+                if (live) {
+                    // w_j x_j as one packed bf16x2 multiply per element pair
+                    const __nv_bfloat162 w2 = __float2bfloat162_rn(__expf(cs_last - cs) * dtv);
+                    const uint8_t* src = smem + kXRing + ((k + 1) % 3) * kRegion;
+                    uint8_t* dst = smem + kXs;
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    *reinterpret_cast<uint4*>(dst + swz(r, half * 4 + c4)) =
-                        make_uint4(yp[4 * c4], yp[4 * c4 + 1], yp[4 * c4 + 2], yp[4 * c4 + 3]);
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int c = half * 4 + c4;
+                        uint4 uv = *reinterpret_cast<const uint4*>(src + swz(r, c));
+                        __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&uv);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) e[j] = __hmul2(e[j], w2);
+                        *reinterpret_cast<uint4*>(dst + swz(r, c)) = uv;
+                    }
+                    fence_proxy_async();
+                    mbar_arrive(bar(BAR_XS));
+                }
             }
-            fence_proxy_async();
-            if (!live || *s_abort) s_ystop[s ^ 1] = 1;
-            group_bar(3);
-            if (leader && !s_ystop[s ^ 1]) {
-                tma_store_4d(&prm.tm_y, sbase + kYst, 0, hd, t0, bi);
-                bulk_commit();
-            }
+            cs_last_prev = cs_last;
         }
-        if (leader) bulk_wait0();
         if (!stopped && live && !*s_abort && prm.hf) {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) prm.hf[hbase + (size_t)(p0 + k) * kN + r] = Hs[k];
+            for (int j = 0; j < 32; ++j) prm.hf[hbase + (size_t)(p0 + j) * kN + r] = Hs[j];
         }
     }
 
     // ================================================================ teardown
-    // The MMA lane has seen its final commit land, the producer its last loads, and the
-    // state group its y stores; only then is the TMEM released.
+    // The MMA lane has seen its final commit land and the producer its last loads; only
+    // then is the TMEM released.
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -672,7 +747,6 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     memset(&prm, 0, sizeof(prm));
     int st;
     if ((st = make_map(&prm.tm_x, x, kP, H, T, b)) != SSD_OK) return st;
-    if ((st = make_map(&prm.tm_y, y, kP, H, T, b)) != SSD_OK) return st;
     if ((st = make_map(&prm.tm_B, Bm, kN, G, T, b)) != SSD_OK) return st;
     if ((st = make_map(&prm.tm_C, Cm, kN, G, T, b)) != SSD_OK) return st;
     prm.dt = dt;
@@ -680,6 +754,7 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     prm.D = D;
     prm.h0 = h0;
     prm.hf = hf;
+    prm.y = static_cast<__nv_bfloat16*>(y);
     prm.status = reinterpret_cast<int*>(ws);
     prm.T = T;
     prm.H = H;
