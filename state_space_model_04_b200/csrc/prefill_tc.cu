@@ -459,7 +459,9 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 tc_fence_after();
                 issue_y(k);
                 if (k + 1 < nblk) {
-                    ok = wt(BAR_H, (k + 1) & 1, 5);
+                    // C H^T buffer (k+1) & 1 was last read (with Y) for block k - 1
+                    ok = wt(BAR_H, (k + 1) & 1, 5) &&
+                         (k < 1 || wt(BAR_YFREE0 + ((k + 1) & 1), ((k - 1) >> 1) & 1, 19));
                     if (!ok) break;
                     tc_fence_after();
                     issue_yst(k + 1);
@@ -530,7 +532,9 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 // chunk by chunk; C B^T is released as soon as the last chunk has been read
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
-                    const int c = half + 2 * cc;
+                    // a diagonal first chunk goes second (its partner is all zeros and needs no
+                    // load), so every warp releases C B^T after one load and one chunk's math
+                    const int c = (half == q) ? half + 2 * (1 - cc) : half + 2 * cc;
                     uint32_t raw[32];
                     if (c <= q) {
                         SSD_TMEM_LD32(tmem + lane_addr + kColCB + c * 32, raw);
@@ -573,8 +577,9 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 if (u >= 1) live = warp_wait(bar(BAR_G2DONE), (u - 1) & 1, s_abort, prm.status, 12);
                 if (live) {
                     tc_fence_after();
-                    SSD_TMEM_ST16(tmem + lane_addr + kColP + half * 16, pk[0]);
-                    SSD_TMEM_ST16(tmem + lane_addr + kColP + (half + 2) * 16, pk[1]);
+                    const int cfirst = (half == q) ? half + 2 : half;
+                    SSD_TMEM_ST16(tmem + lane_addr + kColP + cfirst * 16, pk[0]);
+                    SSD_TMEM_ST16(tmem + lane_addr + kColP + (2 * half + 2 - cfirst) * 16, pk[1]);
                     tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(bar(BAR_SCORES));
