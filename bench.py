@@ -145,6 +145,55 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------- ranks
+class Ranks:
+    """One process per GPU, launched by torchrun: rank and world size from the launcher's
+    environment, a barrier, and the max over ranks of a device-timed duration.  Ranks run
+    independent batches (the prefill's (sequence, head) problems never interact), so the
+    only collectives are the timing barrier and this max.  backend "nccl" on GPUs; the
+    CPU tests use "gloo" with the same code."""
+
+    def __init__(self, backend="nccl", device=None, timeout_s=120):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device
+        self.dist = None
+        if self.world > 1:
+            from datetime import timedelta
+            import torch.distributed as dist
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s), **kw)
+            self.dist = dist
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, v):
+        if self.dist is None:
+            return float(v)
+        import torch
+        t = torch.tensor([float(v)], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def rank_seed(rank, base=2):
+    """Seed of a rank's synthetic batch: every rank draws its own sequences."""
+    return base + 1000 * rank
+
+
+def job_rate(units_per_rank, world, ms_max):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (ms_max * 1e-3)
+
+
 # ----------------------------------------------------------------------------- helpers
 def sha_prefix(path):
     with open(path, "rb") as f:
@@ -250,36 +299,22 @@ def main():
         return run_reference(args)
 
     import torch
-    import torch.distributed as dist
     import state_space_model_04_b200 as ssd
     from ssd_inputs import make_config
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     pk, pk_kind = peaks()
     stream = torch.cuda.current_stream()
 
     # ---------------- prefill inputs (seeded per rank: independent batches)
     PB = args.prefill_batch
-    case = make_config("mamba2_2p7b_layer", seed=2 + 1000 * rank, b=PB)
+    case = make_config("mamba2_2p7b_layer", seed=rank_seed(rank), b=PB)
     def bf(bits):
         return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
     host = {"x": bf(case.x_bits), "B": bf(case.B_bits), "C": bf(case.C_bits),
@@ -318,8 +353,8 @@ def main():
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
     flops = prefill_flops(PB, PT, PH, PP, PN, PG, PL)
     pbytes = prefill_bytes(PB, PT, PH, PP, PN, PG)
-    tflops = flops * world / (ms * 1e-3) / 1e12
-    tokens_s = PB * PT * world / (ms * 1e-3)
+    tflops = job_rate(flops, world, ms) / 1e12
+    tokens_s = job_rate(PB * PT, world, ms)
 
     # dominant kernel: the one with the largest summed event time in the timed region
     dom = max(kt.items(), key=lambda kv: kv[1][1])
@@ -368,7 +403,7 @@ def main():
     ms_e2e = max_over_ranks(e2[0].elapsed_time(e2[1]) / args.steps)
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = y.numel() * y.element_size() + hf.numel() * hf.element_size()
-    e2e = {"value": flops * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+    e2e = {"value": job_rate(flops, world, ms_e2e) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
 
     # ---------------- cached decode (state from this prefill's final state)
@@ -399,8 +434,7 @@ def main():
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
                 "clocks": clk, "decode": decode}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
@@ -442,7 +476,7 @@ def bench_decode(ssd, torch, dev, stream, case, hf, b, args, clocks, barrier, ma
     barrier()
     ms = max_over_ranks(ev[0].elapsed_time(ev[1]))
     steps = launches_timed * steps_per_launch
-    sps = steps * world / (ms * 1e-3)
+    sps = job_rate(steps, world, ms)
     byt = decode_bytes_per_step(DL, b, DH, DP, DN, DG)
     gbs = byt * sps / 1e9
     ok = bool(torch.isfinite(h).all().item())
