@@ -111,6 +111,16 @@ SSD_API int ssd_prefill(int b, int T, int H, int P, int N, int G, int chunk, int
  * check), then clears it.  Each ssd_prefill call resets the status word first. */
 SSD_API int ssd_prefill_check(void* workspace, void* stream);
 
+/* Failure-detection test hook.  Arms a one-shot fault for the next ssd_prefill in this
+ * process that takes the tensor-core path (bf16, P = 64, N = 128): its TMA producer issues
+ * no loads, so every consumer's bounded wait runs out after `wait_limit_ns` (instead of the
+ * default 2 s), the kernel records SSD_ERR_TIMEOUT with the site of the first expired wait,
+ * drains, frees its tensor memory and exits; ssd_prefill_check then returns
+ * SSD_ERR_TIMEOUT and the CUDA context stays usable.  The y and h_final of that call are
+ * undefined.  Nothing faults, traps or spins without a limit.
+ * Errors: SSD_ERR_INVALID_ARG if wait_limit_ns is outside [1e6, 1e10] (1 ms .. 10 s). */
+SSD_API int ssd_debug_starve_next_prefill(unsigned long long wait_limit_ns);
+
 /* ------------------------------------------------------------------------------------
  * Cached decode step  ([CF-SSD] O(1) caching section)
  *

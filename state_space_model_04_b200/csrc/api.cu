@@ -26,6 +26,7 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
                       const void* Cm, const float* D, const float* h0, void* y, float* hf, void* ws,
                       cudaStream_t s);
 int prefill_tc_status(void* ws, cudaStream_t s);
+void prefill_tc_starve_next(unsigned long long wait_ns);
 size_t decode_workspace_bytes(int layers, int b, int G);
 int launch_decode_step(int layers, int b, int H, int N, int G, int act, int io, float* h,
                        float* conv_state, const void* xbc, const float* dt, const float* A,
@@ -202,6 +203,14 @@ size_t ssd_prefill_workspace_size(int b, int T, int H, int P, int N, int G, int 
     if (check_prefill_shape(b, T, H, P, N, G, chunk, io_dtype) != SSD_OK) return 0;
     if (b == 0 || T == 0) return 0;
     return prefill_ws_bytes(b, T, H, P, N, chunk, io_dtype);
+}
+
+int ssd_debug_starve_next_prefill(unsigned long long wait_limit_ns) {
+    g_detail[0] = 0;
+    if (wait_limit_ns < 1000000ull || wait_limit_ns > 10000000000ull)
+        return set_error(SSD_ERR_INVALID_ARG, "wait_limit_ns %llu outside [1e6, 1e10]", wait_limit_ns);
+    prefill_tc_starve_next(wait_limit_ns);
+    return SSD_OK;
 }
 
 int ssd_prefill_check(void* workspace, void* stream) {

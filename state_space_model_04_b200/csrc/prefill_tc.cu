@@ -40,6 +40,7 @@
 // SSD_ERR_TIMEOUT in the status word, each group stops at a point all its threads reach
 // together, in-flight copies and MMAs are drained, the TMEM is released and the kernel
 // returns (no trap, no endless loop).
+#include <atomic>
 #include "common.cuh"
 
 #include <cuda.h>
@@ -111,7 +112,12 @@ struct TcParams {
     __nv_bfloat16* y;
     int* status;
     int T, H, G, nblk;
+    unsigned long long wait_ns;  // limit of every bounded wait
+    int starve;                  // failure-detection test: the producer issues no loads
 };
+
+// per-CTA copy of the wait limit, set before the first wait
+__shared__ unsigned long long s_wait_ns;
 
 // ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -164,7 +170,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     while (true) {
         if (mbar_try_sleep(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > s_wait_ns) {
             *abort_flag = 1;
             atomicCAS(status, 0, SSD_ERR_TIMEOUT | (where << 8));
             return false;
@@ -180,7 +186,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 // Drain: bounded wait that never sets the abort flag (used on the way out).
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
     const unsigned long long t0 = globaltimer();
-    while (!mbar_try(bar, parity) && globaltimer() - t0 < kWaitLimitNs) {
+    while (!mbar_try(bar, parity) && globaltimer() - t0 < s_wait_ns) {
     }
 }
 
@@ -343,6 +349,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             mbar_init(bar(i), group ? kGroupThreads : 1);
         }
         *s_abort = misaligned ? 1 : 0;
+        s_wait_ns = prm.wait_ns;
         s_ystop[0] = s_ystop[1] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -358,7 +365,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 
     if (warp == 0) {
         // ================================================================ TMA producer
-        if (lane == 0 && !*s_abort) {
+        if (lane == 0 && !*s_abort && !prm.starve) {
             int issued = 0;
             for (int u = 0; u < nblk; ++u) {
                 const int s2 = u & 1, s3 = u % 3;
@@ -745,6 +752,11 @@ bool prefill_tc_supported(int P, int N, int io) { return io == SSD_BF16 && P == 
 
 size_t prefill_tc_workspace_bytes() { return 256; }
 
+namespace {
+std::atomic<unsigned long long> g_starve_ns{0};
+}
+void prefill_tc_starve_next(unsigned long long wait_ns) { g_starve_ns.store(wait_ns); }
+
 int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt, const float* A, const void* Bm,
                       const void* Cm, const float* D, const float* h0, void* y, float* hf, void* ws,
                       cudaStream_t s) {
@@ -765,6 +777,9 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     prm.H = H;
     prm.G = G;
     prm.nblk = (T + kBlk - 1) / kBlk;
+    const unsigned long long starve_ns = g_starve_ns.exchange(0);
+    prm.starve = starve_ns != 0;
+    prm.wait_ns = starve_ns ? starve_ns : kWaitLimitNs;
     SSD_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), s));
     SSD_CUDA_TRY(cudaFuncSetAttribute(ssd_prefill_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kSmemBytes));

@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill.restype = _i
         L.ssd_prefill_check.argtypes = [_vp, _vp]
         L.ssd_prefill_check.restype = _i
+        L.ssd_debug_starve_next_prefill.argtypes = [ctypes.c_ulonglong]
+        L.ssd_debug_starve_next_prefill.restype = _i
         L.ssd_decode_workspace_size.argtypes = [_i] * 3
         L.ssd_decode_workspace_size.restype = _sz
         L.ssd_decode_step.argtypes = [_i] * 9 + [_vp] * 10 + [_sz, _vp]
@@ -182,6 +184,12 @@ def prefill(x, dt, A, B, C, D, chunk=256, h0=None, y=None, h_final=None, workspa
 def prefill_check(workspace, stream=None):
     """Synchronise and raise if the last prefill on `workspace` recorded a device-side error."""
     _check(lib().ssd_prefill_check(_ptr(workspace), _stream(stream)), "ssd_prefill_check")
+
+
+def debug_starve_next_prefill(wait_limit_s=0.1):
+    """Failure-detection test hook: the next tensor-core prefill issues no loads, so its
+    bounded waits expire after `wait_limit_s` and prefill_check raises SSD_ERR_TIMEOUT."""
+    _check(lib().ssd_debug_starve_next_prefill(int(wait_limit_s * 1e9)), "ssd_debug_starve_next_prefill")
 
 
 def decode_workspace_size(layers, b, G) -> int:

@@ -156,3 +156,10 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         ssd.prefill(x, torch.zeros(1, 64, 4), torch.zeros(4), torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16),
                     torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16), torch.zeros(4))
+
+
+def test_starve_hook_rejects_out_of_range_limits():
+    import state_space_model_04_b200 as ssd
+    L = ssd.lib()
+    assert L.ssd_debug_starve_next_prefill(999_999) == 1
+    assert L.ssd_debug_starve_next_prefill(10_000_000_001) == 1

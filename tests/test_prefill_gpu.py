@@ -190,6 +190,27 @@ def test_weak_decay_long_memory():
     _full_check(case)
 
 
+def test_bounded_wait_timeout_reports_status_and_context_survives():
+    """Failure detection without a fault: the armed test hook starves the next fused prefill
+    of its inputs; every wait gives up after 0.1 s, the call reports SSD_ERR_TIMEOUT with a
+    wait site, and the next prefill on the same context is correct."""
+    case = make_prefill(1, 512, 2, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=16)
+    t = prefill_inputs(case)
+    ws = torch.empty(ssd.prefill_workspace_size(1, 512, 2, 64, 128, 1, 256, ssd.SSD_BF16), dtype=torch.uint8,
+                     device="cuda")
+    ssd.debug_starve_next_prefill(0.1)
+    ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=256, h0=t["h0"], workspace=ws)
+    with pytest.raises(ssd.SSDError) as e:
+        ssd.prefill_check(ws)
+    assert e.value.status == 4 and "wait site" in str(e.value)   # SSD_ERR_TIMEOUT
+    ssd.prefill_check(ws)                                        # the status word was cleared
+    y, hf = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=256, h0=t["h0"], workspace=ws)
+    ssd.prefill_check(ws)
+    y_ref, hf_ref = oracle_subset(case, [0], [0, 1])
+    check(_np(y), y_ref, "bf16", "y after timeout")
+    check(_np(hf), hf_ref, "bf16", "h_final after timeout")
+
+
 def test_in_place_state_resume():
     """h_final may alias h0 exactly (in-place cache update)."""
     case = make_prefill(1, 512, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=14)
