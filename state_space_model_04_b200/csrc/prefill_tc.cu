@@ -17,7 +17,7 @@
 // shorter segment, identical in exact arithmetic.
 //
 //   warp 0       TMA producer: C and B (two 64-column 128B-swizzled boxes each) into a
-//                2-slot ring, X into a 3-slot ring
+//                2-slot ring, X into a 2-slot ring
 //   warp 1       TMEM owner and MMA issuer (one lane).  Iteration k:
 //                  Y(k)      = P(k) X(k)      (M=128 i, N=64 p,  K=128 j)  TS, P in TMEM
 //                  CB(k+1)   = C B^T          (M=128 i, N=128 j, K=128 n)  SS
@@ -25,11 +25,12 @@
 //                  S(k+1)^T  = B^T (w o X)    (M=128 n, N=64 p,  K=128 j)  SS
 //                so C and B of a block are dead within one iteration and the next
 //                block's loads run a full iteration ahead of their use.
-//   warps 2-9    "scores" group (2 warps per TMEM lane quadrant): prefix sum of dt*A and
-//                P = bf16(CB o L), written back into TMEM as the A operand of P X
-//   warps 10-17  "state" group (2 warps per quadrant): prefix sums, w o X into shared
-//                memory, H <- exp(cs_last) H + S (fp32 registers) with its bf16 copy for
-//                C H^T, and y = Y + exp(cs_i) Yst stored straight from registers
+//   warps 2-9    "scores" group (2 warps per TMEM lane quadrant): P = bf16(CB o L),
+//                written back into TMEM as the A operand of P X; y = Y + exp(cs_i) Yst
+//                into a swizzled shared tile that one lane stores with a TMA tensor store
+//   warps 10-17  "state" group (2 warps per quadrant): prefix sums of dt*A, the decay
+//                arrays, w o X into shared memory, H <- exp(cs_last) H + S (fp32
+//                registers) with its bf16 copy for C H^T
 //
 // Decay arithmetic.  Below the 32x32 diagonal sub-blocks the decay factorises exactly
 // as exp(cs_i - cs_e) * exp(cs_e - cs_j) with e the last token of j's 32-token group
@@ -61,10 +62,11 @@ constexpr uint32_t kRegion = kBlk * 128;             // one [128 rows][64 bf16] 
 constexpr uint32_t kCBSlot = 4 * kRegion;            // C (2 regions: n 0..63, 64..127) then B (2)
 constexpr uint32_t kSlotC = 0;
 constexpr uint32_t kSlotB = 2 * kRegion;
-constexpr uint32_t kXRing = 2 * kCBSlot;             // 3 X slots of one region
-constexpr uint32_t kXs = kXRing + 3 * kRegion;       // w o X
+constexpr uint32_t kXRing = 2 * kCBSlot;             // 2 X slots of one region
+constexpr uint32_t kXs = kXRing + 2 * kRegion;       // w o X
 constexpr uint32_t kSH = kXs + kRegion;              // bf16 H^T [n][p]
-constexpr uint32_t kSmall = kSH + kRegion;           // barriers and per-token scalars
+constexpr uint32_t kYStage = kSH + kRegion;          // bf16 y tile [t][p] for the TMA store
+constexpr uint32_t kSmall = kYStage + kRegion;       // barriers and per-token scalars
 constexpr uint32_t kSmallBytes = 4096;
 constexpr uint32_t kSmemBytes = kSmall + kSmallBytes;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -83,9 +85,9 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 enum {
     BAR_FULLCB = 0,   // [2] C,B landed
     BAR_EMPTYCB = 2,  // [2] C,B slot released by the MMAs
-    BAR_FULLX = 4,    // [3] X landed
-    BAR_EMPTYX = 7,   // [3] X slot released
-    BAR_CBFULL = 10,  // C B^T accumulated
+    BAR_FULLX = 4,    // [2] X landed
+    BAR_EMPTYX = 6,   // [2] X slot released
+    BAR_CBFULL = 8,   // C B^T accumulated
     BAR_CBFREE,       // scores group has read C B^T            (256 arrivals)
     BAR_XS,           // state group has written w o X          (256)
     BAR_ACCS,         // S^T accumulated (and w o X read)
@@ -96,7 +98,9 @@ enum {
     BAR_G2DONE,       // P X accumulated (and P read)
     BAR_YFREE0,       // [2] scores group has read Y and C H^T of the slot (256)
     BAR_PREP0 = BAR_YFREE0 + 2,  // [2] state group has published a block's decay arrays (256)
-    BAR_DONE = BAR_PREP0 + 2,
+    BAR_YSTAGED = BAR_PREP0 + 2,  // scores group has written the y tile (256)
+    BAR_STAGEFREE,                // the TMA store has read the y tile (1)
+    BAR_DONE,
     BAR_COUNT
 };
 
@@ -104,6 +108,7 @@ struct TcParams {
     CUtensorMap tm_x;
     CUtensorMap tm_B;
     CUtensorMap tm_C;
+    CUtensorMap tm_y;
     const float* dt;
     const float* A;
     const float* D;
@@ -197,6 +202,15 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm,
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
+// y tile: shared -> global through the async proxy (rows past T are clipped by the map)
+__device__ __forceinline__ void tma_store_4d(uint32_t src, const CUtensorMap* tm, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(tm)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -345,7 +359,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         for (int i = 0; i < BAR_COUNT; ++i) {
             const bool group = (i == BAR_CBFREE || i == BAR_XS || i == BAR_SFREE || i == BAR_H ||
                                 i == BAR_SCORES || i == BAR_YFREE0 || i == BAR_YFREE0 + 1 || i == BAR_PREP0 ||
-                                i == BAR_PREP0 + 1);
+                                i == BAR_PREP0 + 1 || i == BAR_YSTAGED);
             mbar_init(bar(i), group ? kGroupThreads : 1);
         }
         *s_abort = misaligned ? 1 : 0;
@@ -368,7 +382,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         if (lane == 0 && !*s_abort && !prm.starve) {
             int issued = 0;
             for (int u = 0; u < nblk; ++u) {
-                const int s2 = u & 1, s3 = u % 3;
+                const int s2 = u & 1;
                 const int t0 = u * kBlk;
                 if (u >= 2 && !mbar_wait(bar(BAR_EMPTYCB + s2), ((u - 2) >> 1) & 1, s_abort, prm.status, 1)) break;
                 const uint32_t fcb = bar(BAR_FULLCB + s2);
@@ -378,13 +392,13 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 tma_load_4d(slot + kSlotC + kRegion, &prm.tm_C, fcb, 64, g, t0, bi);
                 tma_load_4d(slot + kSlotB, &prm.tm_B, fcb, 0, g, t0, bi);
                 tma_load_4d(slot + kSlotB + kRegion, &prm.tm_B, fcb, 64, g, t0, bi);
-                if (u >= 3 && !mbar_wait(bar(BAR_EMPTYX + s3), ((u - 3) / 3) & 1, s_abort, prm.status, 2)) {
+                if (u >= 2 && !mbar_wait(bar(BAR_EMPTYX + s2), ((u - 2) >> 1) & 1, s_abort, prm.status, 2)) {
                     issued = -(u + 1);  // C,B of block u issued, X not
                     break;
                 }
-                const uint32_t fx = bar(BAR_FULLX + s3);
+                const uint32_t fx = bar(BAR_FULLX + s2);
                 mbar_expect_tx(fx, kRegion);
-                tma_load_4d(sbase + kXRing + s3 * kRegion, &prm.tm_x, fx, 0, hd, t0, bi);
+                tma_load_4d(sbase + kXRing + s2 * kRegion, &prm.tm_x, fx, 0, hd, t0, bi);
                 issued = u + 1;
             }
             // loads nobody may have waited for must land before the CTA exits
@@ -392,8 +406,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             const int nx = issued < 0 ? -issued - 1 : issued;
             for (int u = ncb - 2; u < ncb; ++u)
                 if (u >= 0) mbar_drain(bar(BAR_FULLCB + (u & 1)), (u >> 1) & 1);
-            for (int u = nx - 3; u < nx; ++u)
-                if (u >= 0) mbar_drain(bar(BAR_FULLX + u % 3), (u / 3) & 1);
+            for (int u = nx - 2; u < nx; ++u)
+                if (u >= 0) mbar_drain(bar(BAR_FULLX + (u & 1)), (u >> 1) & 1);
         }
     } else if (warp == 1) {
         // ================================================================ MMA issuer
@@ -436,12 +450,12 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             mma_commit_w(bar(BAR_EMPTYCB + (u & 1)));
         };
         auto issue_y = [&](int k) {  // Y_k = P_k X_k; then X of block k is dead
-            const uint64_t dX = sdesc(sbase + kXRing + (k % 3) * kRegion, kRegion, 1024);
+            const uint64_t dX = sdesc(sbase + kXRing + (k & 1) * kRegion, kRegion, 1024);
 #pragma unroll
             for (int kk = 0; kk < kBlk / 16; ++kk)
                 mma_ts_w(tmem + kColY + (k & 1) * 64, tmem + kColP + kk * 8, dX + kk * 128, id_y, kk > 0);
             mma_commit_w(bar(BAR_G2DONE));
-            mma_commit_w(bar(BAR_EMPTYX + k % 3));
+            mma_commit_w(bar(BAR_EMPTYX + (k & 1)));
         };
         bool ok = __all_sync(0xffffffffu, !*s_abort);
         if (ok) {
@@ -460,7 +474,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                     issue_cb(k + 1);
                 }
                 // Y and C H^T buffers k & 1 were last read for block k - 2
-                ok = wt(BAR_FULLX + k % 3, (k / 3) & 1, 8) && wt(BAR_SCORES, k & 1, 9) &&
+                ok = wt(BAR_FULLX + (k & 1), (k >> 1) & 1, 8) && wt(BAR_SCORES, k & 1, 9) &&
                      (k < 2 || wt(BAR_YFREE0 + (k & 1), ((k - 2) >> 1) & 1, 10));
                 if (!ok) break;
                 tc_fence_after();
@@ -489,7 +503,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
         const float Dh = prm.D[hd];
         const int p0 = half * 32;  // this warp's 32 of the 64 p columns of the output
-        // y(k) = Y(k) + exp(cs_i) Yst(k) for row r, columns [p0, p0 + 32), straight to global.
+        // y(k) = Y(k) + exp(cs_i) Yst(k) for row r, columns [p0, p0 + 32), into the swizzled
+        // y tile; warp 2 stores the tile with one TMA store once all 256 rows-halves are in.
         // exp(cs_i) is carried in a register: by now the state group may have republished
         // the per-token arrays of block k's slot.
         auto store_y = [&](int k, float ei) {
@@ -508,13 +523,28 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             }
             tc_fence_before();
             mbar_arrive(bar(BAR_YFREE0 + (k & 1)));
-            const int tok = k * kBlk + r;
-            if (tok < T) {
-                uint4* dst = reinterpret_cast<uint4*>(prm.y + (((size_t)bi * T + tok) * H + hd) * kP + p0);
+            // the previous tile must have been read out by its TMA store
+            bool ok = k < 1 || warp_wait(bar(BAR_STAGEFREE), (k - 1) & 1, s_abort, prm.status, 20);
+            if (ok) {
+                uint8_t* dst = smem + kYStage;
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4)
-                    dst[c4] = make_uint4(yp[4 * c4], yp[4 * c4 + 1], yp[4 * c4 + 2], yp[4 * c4 + 3]);
+                    *reinterpret_cast<uint4*>(dst + swz(r, half * 4 + c4)) =
+                        make_uint4(yp[4 * c4], yp[4 * c4 + 1], yp[4 * c4 + 2], yp[4 * c4 + 3]);
+                fence_proxy_async();
+                mbar_arrive(bar(BAR_YSTAGED));
+                if (warp == 2) {
+                    ok = warp_wait(bar(BAR_YSTAGED), k & 1, s_abort, prm.status, 21);
+                    if (ok && lane == 0) {
+                        tma_store_4d(sbase + kYStage, &prm.tm_y, 0, hd, k * kBlk, bi);
+                        bulk_commit();
+                        bulk_wait_read0();
+                        mbar_arrive(bar(BAR_STAGEFREE));
+                    }
+                    __syncwarp();
+                }
             }
+            return ok;
         };
         bool live = __all_sync(0xffffffffu, !*s_abort);
         float ei_prev = 0.f;  // exp(cs_i) of the previous block
@@ -592,13 +622,15 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                     mbar_arrive(bar(BAR_SCORES));
                 }
                 // the previous block's output, once P is published (P X of block u-1 is done)
-                if (live && u >= 1) store_y(u - 1, ei_prev);
+                if (live && u >= 1) live = store_y(u - 1, ei_prev);
             }
             ei_prev = ei_cur;
         }
         // output of the last block
         if (live && nblk > 0) live = warp_wait(bar(BAR_G2DONE), (nblk - 1) & 1, s_abort, prm.status, 18);
-        if (live && nblk > 0) store_y(nblk - 1, ei_prev);
+        if (live && nblk > 0) live = store_y(nblk - 1, ei_prev);
+        // the tile stores must be complete before the CTA's shared memory goes away
+        if (warp == 2 && lane == 0) bulk_wait0();
     } else {
         // ================================================================ state group
         const int q = warp & 3, half = (warp - 10) >> 2;
@@ -681,11 +713,11 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             // ---- w o X of block k+1 (after the H hand-off: C H^T needs H sooner than the
             //      state MMA needs w o X)
             if (live && k + 1 < nblk) {
-                live = warp_wait(bar(BAR_FULLX + (k + 1) % 3), ((k + 1) / 3) & 1, s_abort, prm.status, 14);
+                live = warp_wait(bar(BAR_FULLX + ((k + 1) & 1)), ((k + 1) >> 1) & 1, s_abort, prm.status, 14);
                 if (live) {
                     // w_j x_j as one packed bf16x2 multiply per element pair
                     const __nv_bfloat162 w2 = __float2bfloat162_rn(__expf(cs_last - cs) * dtv);
-                    const uint8_t* src = smem + kXRing + ((k + 1) % 3) * kRegion;
+                    const uint8_t* src = smem + kXRing + ((k + 1) & 1) * kRegion;
                     uint8_t* dst = smem + kXs;
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
@@ -766,6 +798,7 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     if ((st = make_map(&prm.tm_x, x, kP, H, T, b)) != SSD_OK) return st;
     if ((st = make_map(&prm.tm_B, Bm, kN, G, T, b)) != SSD_OK) return st;
     if ((st = make_map(&prm.tm_C, Cm, kN, G, T, b)) != SSD_OK) return st;
+    if ((st = make_map(&prm.tm_y, y, kP, H, T, b)) != SSD_OK) return st;
     prm.dt = dt;
     prm.A = A;
     prm.D = D;
