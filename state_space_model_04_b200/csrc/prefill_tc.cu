@@ -17,7 +17,7 @@
 // shorter segment, identical in exact arithmetic.
 //
 //   warp 0       TMA producer: C and B (two 64-column 128B-swizzled boxes each) into a
-//                2-slot ring, X into a 2-slot ring
+//                2-slot ring, X into a 3-slot ring (slot k % 3 later holds y of block k)
 //   warp 1       TMEM owner and MMA issuer (one lane).  Iteration k:
 //                  Y(k)      = P(k) X(k)      (M=128 i, N=64 p,  K=128 j)  TS, P in TMEM
 //                  CB(k+1)   = C B^T          (M=128 i, N=128 j, K=128 n)  SS
@@ -27,10 +27,12 @@
 //                block's loads run a full iteration ahead of their use.
 //   warps 2-9    "scores" group (2 warps per TMEM lane quadrant): P = bf16(CB o L),
 //                written back into TMEM as the A operand of P X; y = Y + exp(cs_i) Yst
-//                into a swizzled shared tile that one lane stores with a TMA tensor store
+//                into a swizzled shared tile (the block's dead X slot)
 //   warps 10-17  "state" group (2 warps per quadrant): prefix sums of dt*A, the decay
 //                arrays, w o X into shared memory, H <- exp(cs_last) H + S (fp32
 //                registers) with its bf16 copy for C H^T
+//   warp 18      y store: one TMA tensor store per block, then the X slot goes back to
+//                the producer
 //
 // Decay arithmetic.  Below the 32x32 diagonal sub-blocks the decay factorises exactly
 // as exp(cs_i - cs_e) * exp(cs_e - cs_j) with e the last token of j's 32-token group
@@ -54,7 +56,7 @@ constexpr int kBlk = 128;    // tokens per block = MMA M
 constexpr int kP = 64;       // head dim
 constexpr int kN = 128;      // state size
 constexpr int kGroupThreads = 256;  // threads per epilogue group
-constexpr int kThreads = 64 + 2 * kGroupThreads;
+constexpr int kThreads = 64 + 2 * kGroupThreads + 32;  // + the y-store warp
 constexpr float kLog2e = 1.4426950408889634f;
 
 // shared memory map (bytes from a 1024-aligned base)
@@ -62,11 +64,11 @@ constexpr uint32_t kRegion = kBlk * 128;             // one [128 rows][64 bf16] 
 constexpr uint32_t kCBSlot = 4 * kRegion;            // C (2 regions: n 0..63, 64..127) then B (2)
 constexpr uint32_t kSlotC = 0;
 constexpr uint32_t kSlotB = 2 * kRegion;
-constexpr uint32_t kXRing = 2 * kCBSlot;             // 2 X slots of one region
-constexpr uint32_t kXs = kXRing + 2 * kRegion;       // w o X
+constexpr uint32_t kXRing = 2 * kCBSlot;             // 3 X slots of one region; slot k % 3 holds
+                                                     // X(k), then the bf16 y tile of block k
+constexpr uint32_t kXs = kXRing + 3 * kRegion;       // w o X
 constexpr uint32_t kSH = kXs + kRegion;              // bf16 H^T [n][p]
-constexpr uint32_t kYStage = kSH + kRegion;          // bf16 y tile [t][p] for the TMA store
-constexpr uint32_t kSmall = kYStage + kRegion;       // barriers and per-token scalars
+constexpr uint32_t kSmall = kSH + kRegion;           // barriers and per-token scalars
 constexpr uint32_t kSmallBytes = 4096;
 constexpr uint32_t kSmemBytes = kSmall + kSmallBytes;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -85,9 +87,9 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 enum {
     BAR_FULLCB = 0,   // [2] C,B landed
     BAR_EMPTYCB = 2,  // [2] C,B slot released by the MMAs
-    BAR_FULLX = 4,    // [2] X landed
-    BAR_EMPTYX = 6,   // [2] X slot released
-    BAR_CBFULL = 8,   // C B^T accumulated
+    BAR_FULLX = 4,    // [3] X landed
+    BAR_EMPTYX = 7,   // [3] X slot released (its y tile has been read by the TMA store)
+    BAR_CBFULL = 10,  // C B^T accumulated
     BAR_CBFREE,       // scores group has read C B^T            (256 arrivals)
     BAR_XS,           // state group has written w o X          (256)
     BAR_ACCS,         // S^T accumulated (and w o X read)
@@ -98,9 +100,8 @@ enum {
     BAR_G2DONE,       // P X accumulated (and P read)
     BAR_YFREE0,       // [2] scores group has read Y and C H^T of the slot (256)
     BAR_PREP0 = BAR_YFREE0 + 2,  // [2] state group has published a block's decay arrays (256)
-    BAR_YSTAGED = BAR_PREP0 + 2,  // scores group has written the y tile (256)
-    BAR_STAGEFREE,                // the TMA store has read the y tile (1)
-    BAR_DONE,
+    BAR_YSTAGED = BAR_PREP0 + 2,  // [3] scores group has written the y tile into X slot (256)
+    BAR_DONE = BAR_YSTAGED + 3,
     BAR_COUNT
 };
 
@@ -359,7 +360,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         for (int i = 0; i < BAR_COUNT; ++i) {
             const bool group = (i == BAR_CBFREE || i == BAR_XS || i == BAR_SFREE || i == BAR_H ||
                                 i == BAR_SCORES || i == BAR_YFREE0 || i == BAR_YFREE0 + 1 || i == BAR_PREP0 ||
-                                i == BAR_PREP0 + 1 || i == BAR_YSTAGED);
+                                i == BAR_PREP0 + 1 || (i >= BAR_YSTAGED && i < BAR_YSTAGED + 3));
             mbar_init(bar(i), group ? kGroupThreads : 1);
         }
         *s_abort = misaligned ? 1 : 0;
@@ -382,7 +383,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         if (lane == 0 && !*s_abort && !prm.starve) {
             int issued = 0;
             for (int u = 0; u < nblk; ++u) {
-                const int s2 = u & 1;
+                const int s2 = u & 1, s3 = u % 3;
                 const int t0 = u * kBlk;
                 if (u >= 2 && !mbar_wait(bar(BAR_EMPTYCB + s2), ((u - 2) >> 1) & 1, s_abort, prm.status, 1)) break;
                 const uint32_t fcb = bar(BAR_FULLCB + s2);
@@ -392,13 +393,13 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 tma_load_4d(slot + kSlotC + kRegion, &prm.tm_C, fcb, 64, g, t0, bi);
                 tma_load_4d(slot + kSlotB, &prm.tm_B, fcb, 0, g, t0, bi);
                 tma_load_4d(slot + kSlotB + kRegion, &prm.tm_B, fcb, 64, g, t0, bi);
-                if (u >= 2 && !mbar_wait(bar(BAR_EMPTYX + s2), ((u - 2) >> 1) & 1, s_abort, prm.status, 2)) {
+                if (u >= 3 && !mbar_wait(bar(BAR_EMPTYX + s3), ((u - 3) / 3) & 1, s_abort, prm.status, 2)) {
                     issued = -(u + 1);  // C,B of block u issued, X not
                     break;
                 }
-                const uint32_t fx = bar(BAR_FULLX + s2);
+                const uint32_t fx = bar(BAR_FULLX + s3);
                 mbar_expect_tx(fx, kRegion);
-                tma_load_4d(sbase + kXRing + s2 * kRegion, &prm.tm_x, fx, 0, hd, t0, bi);
+                tma_load_4d(sbase + kXRing + s3 * kRegion, &prm.tm_x, fx, 0, hd, t0, bi);
                 issued = u + 1;
             }
             // loads nobody may have waited for must land before the CTA exits
@@ -406,8 +407,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             const int nx = issued < 0 ? -issued - 1 : issued;
             for (int u = ncb - 2; u < ncb; ++u)
                 if (u >= 0) mbar_drain(bar(BAR_FULLCB + (u & 1)), (u >> 1) & 1);
-            for (int u = nx - 2; u < nx; ++u)
-                if (u >= 0) mbar_drain(bar(BAR_FULLX + (u & 1)), (u >> 1) & 1);
+            for (int u = nx - 3; u < nx; ++u)
+                if (u >= 0) mbar_drain(bar(BAR_FULLX + u % 3), (u / 3) & 1);
         }
     } else if (warp == 1) {
         // ================================================================ MMA issuer
@@ -450,12 +451,11 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             mma_commit_w(bar(BAR_EMPTYCB + (u & 1)));
         };
         auto issue_y = [&](int k) {  // Y_k = P_k X_k; then X of block k is dead
-            const uint64_t dX = sdesc(sbase + kXRing + (k & 1) * kRegion, kRegion, 1024);
+            const uint64_t dX = sdesc(sbase + kXRing + (k % 3) * kRegion, kRegion, 1024);
 #pragma unroll
             for (int kk = 0; kk < kBlk / 16; ++kk)
                 mma_ts_w(tmem + kColY + (k & 1) * 64, tmem + kColP + kk * 8, dX + kk * 128, id_y, kk > 0);
             mma_commit_w(bar(BAR_G2DONE));
-            mma_commit_w(bar(BAR_EMPTYX + (k & 1)));
         };
         bool ok = __all_sync(0xffffffffu, !*s_abort);
         if (ok) {
@@ -474,7 +474,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                     issue_cb(k + 1);
                 }
                 // Y and C H^T buffers k & 1 were last read for block k - 2
-                ok = wt(BAR_FULLX + (k & 1), (k >> 1) & 1, 8) && wt(BAR_SCORES, k & 1, 9) &&
+                ok = wt(BAR_FULLX + k % 3, (k / 3) & 1, 8) && wt(BAR_SCORES, k & 1, 9) &&
                      (k < 2 || wt(BAR_YFREE0 + (k & 1), ((k - 2) >> 1) & 1, 10));
                 if (!ok) break;
                 tc_fence_after();
@@ -504,7 +504,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         const float Dh = prm.D[hd];
         const int p0 = half * 32;  // this warp's 32 of the 64 p columns of the output
         // y(k) = Y(k) + exp(cs_i) Yst(k) for row r, columns [p0, p0 + 32), into the swizzled
-        // y tile; warp 2 stores the tile with one TMA store once all 256 rows-halves are in.
+        // y tile in X slot k % 3 (X(k) is dead once P X of block k is done, which every
+        // caller has waited for); the store warp writes the tile out with one TMA store.
         // exp(cs_i) is carried in a register: by now the state group may have republished
         // the per-token arrays of block k's slot.
         auto store_y = [&](int k, float ei) {
@@ -523,28 +524,14 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             }
             tc_fence_before();
             mbar_arrive(bar(BAR_YFREE0 + (k & 1)));
-            // the previous tile must have been read out by its TMA store
-            bool ok = k < 1 || warp_wait(bar(BAR_STAGEFREE), (k - 1) & 1, s_abort, prm.status, 20);
-            if (ok) {
-                uint8_t* dst = smem + kYStage;
+            uint8_t* dst = smem + kXRing + (k % 3) * kRegion;
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    *reinterpret_cast<uint4*>(dst + swz(r, half * 4 + c4)) =
-                        make_uint4(yp[4 * c4], yp[4 * c4 + 1], yp[4 * c4 + 2], yp[4 * c4 + 3]);
-                fence_proxy_async();
-                mbar_arrive(bar(BAR_YSTAGED));
-                if (warp == 2) {
-                    ok = warp_wait(bar(BAR_YSTAGED), k & 1, s_abort, prm.status, 21);
-                    if (ok && lane == 0) {
-                        tma_store_4d(sbase + kYStage, &prm.tm_y, 0, hd, k * kBlk, bi);
-                        bulk_commit();
-                        bulk_wait_read0();
-                        mbar_arrive(bar(BAR_STAGEFREE));
-                    }
-                    __syncwarp();
-                }
-            }
-            return ok;
+            for (int c4 = 0; c4 < 4; ++c4)
+                *reinterpret_cast<uint4*>(dst + swz(r, half * 4 + c4)) =
+                    make_uint4(yp[4 * c4], yp[4 * c4 + 1], yp[4 * c4 + 2], yp[4 * c4 + 3]);
+            fence_proxy_async();
+            mbar_arrive(bar(BAR_YSTAGED + k % 3));
+            return true;
         };
         bool live = __all_sync(0xffffffffu, !*s_abort);
         float ei_prev = 0.f;  // exp(cs_i) of the previous block
@@ -629,9 +616,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         // output of the last block
         if (live && nblk > 0) live = warp_wait(bar(BAR_G2DONE), (nblk - 1) & 1, s_abort, prm.status, 18);
         if (live && nblk > 0) live = store_y(nblk - 1, ei_prev);
-        // the tile stores must be complete before the CTA's shared memory goes away
-        if (warp == 2 && lane == 0) bulk_wait0();
-    } else {
+    } else if (warp < 18) {
         // ================================================================ state group
         const int q = warp & 3, half = (warp - 10) >> 2;
         const int r = q * 32 + lane;  // token row (w o X, y) and state row n (S, H)
@@ -713,11 +698,11 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             // ---- w o X of block k+1 (after the H hand-off: C H^T needs H sooner than the
             //      state MMA needs w o X)
             if (live && k + 1 < nblk) {
-                live = warp_wait(bar(BAR_FULLX + ((k + 1) & 1)), ((k + 1) >> 1) & 1, s_abort, prm.status, 14);
+                live = warp_wait(bar(BAR_FULLX + (k + 1) % 3), ((k + 1) / 3) & 1, s_abort, prm.status, 14);
                 if (live) {
                     // w_j x_j as one packed bf16x2 multiply per element pair
                     const __nv_bfloat162 w2 = __float2bfloat162_rn(__expf(cs_last - cs) * dtv);
-                    const uint8_t* src = smem + kXRing + ((k + 1) & 1) * kRegion;
+                    const uint8_t* src = smem + kXRing + ((k + 1) % 3) * kRegion;
                     uint8_t* dst = smem + kXs;
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
@@ -737,6 +722,24 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         if (!stopped && live && !*s_abort && prm.hf) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) prm.hf[hbase + (size_t)(p0 + j) * kN + r] = Hs[j];
+        }
+    } else {
+        // ================================================================ y-store warp
+        // One lane writes each block's y tile with a TMA store once the scores group has
+        // staged it, waits until the store has read the tile out of shared memory, and
+        // returns the X slot to the producer.  Kept off the scores group's path: a store
+        // queued behind the producer's loads can take microseconds to drain.
+        if (lane == 0 && !*s_abort) {
+            for (int k = 0; k < nblk; ++k) {
+                const int s3 = k % 3;
+                if (!mbar_wait(bar(BAR_YSTAGED + s3), (k / 3) & 1, s_abort, prm.status, 20)) break;
+                tma_store_4d(sbase + kXRing + s3 * kRegion, &prm.tm_y, 0, hd, k * kBlk, bi);
+                bulk_commit();
+                bulk_wait_read0();
+                mbar_arrive(bar(BAR_EMPTYX + s3));
+            }
+            // the stores must be complete before the CTA's shared memory goes away
+            bulk_wait0();
         }
     }
 
