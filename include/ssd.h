@@ -121,6 +121,16 @@ SSD_API int ssd_prefill_check(void* workspace, void* stream);
  * Errors: SSD_ERR_INVALID_ARG if wait_limit_ns is outside [1e6, 1e10] (1 ms .. 10 s). */
 SSD_API int ssd_debug_starve_next_prefill(unsigned long long wait_limit_ns);
 
+/* Test hook for the sequence split of the tensor-core prefill.  With nseg >= 1, every
+ * following tensor-core ssd_prefill (and ssd_prefill_workspace_size) in this process
+ * splits each sequence into min(nseg, ceil(T / 128)) segments of whole 128-token blocks
+ * instead of the count its cost model picks; nseg = 0 restores the cost model.  The
+ * result is the same function either way (only rounding differs): segments after the
+ * first start from the state a scan of the earlier segments' local end states gives.
+ * Not thread-safe against concurrent prefill calls.
+ * Errors: SSD_ERR_INVALID_ARG if nseg < 0. */
+SSD_API int ssd_debug_force_prefill_segments(int nseg);
+
 /* ------------------------------------------------------------------------------------
  * Cached decode step  ([CF-SSD] O(1) caching section)
  *

@@ -21,12 +21,13 @@ int launch_prefill_simt(int b, int T, int H, int N, int G, int L, int io, const 
                         const float* D, const float* h0, void* y, float* hf, void* ws,
                         cudaStream_t s);
 bool prefill_tc_supported(int P, int N, int io);
-size_t prefill_tc_workspace_bytes();
+size_t prefill_tc_workspace_bytes(int b, int T, int H);
 int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt, const float* A, const void* Bm,
                       const void* Cm, const float* D, const float* h0, void* y, float* hf, void* ws,
                       cudaStream_t s);
 int prefill_tc_status(void* ws, cudaStream_t s);
 void prefill_tc_starve_next(unsigned long long wait_ns);
+void prefill_tc_force_segments(int nseg);
 size_t decode_workspace_bytes(int layers, int b, int G);
 int launch_decode_step(int layers, int b, int H, int N, int G, int act, int io, float* h,
                        float* conv_state, const void* xbc, const float* dt, const float* A,
@@ -195,7 +196,7 @@ int ssd_profile_end(ssd_kernel_time* out, int max_entries) {
 static constexpr size_t kStatusBytes = 256;
 
 static size_t prefill_ws_bytes(int b, int T, int H, int P, int N, int chunk, int io) {
-    if (prefill_tc_supported(P, N, io)) return kStatusBytes + prefill_tc_workspace_bytes();
+    if (prefill_tc_supported(P, N, io)) return kStatusBytes + prefill_tc_workspace_bytes(b, T, H);
     return kStatusBytes + prefill_simt_workspace_bytes(b, T, H, N, chunk, io);
 }
 
@@ -210,6 +211,13 @@ int ssd_debug_starve_next_prefill(unsigned long long wait_limit_ns) {
     if (wait_limit_ns < 1000000ull || wait_limit_ns > 10000000000ull)
         return set_error(SSD_ERR_INVALID_ARG, "wait_limit_ns %llu outside [1e6, 1e10]", wait_limit_ns);
     prefill_tc_starve_next(wait_limit_ns);
+    return SSD_OK;
+}
+
+int ssd_debug_force_prefill_segments(int nseg) {
+    g_detail[0] = 0;
+    if (nseg < 0) return set_error(SSD_ERR_INVALID_ARG, "nseg %d is negative", nseg);
+    prefill_tc_force_segments(nseg);
     return SSD_OK;
 }
 

@@ -43,7 +43,9 @@
 // SSD_ERR_TIMEOUT in the status word, each group stops at a point all its threads reach
 // together, in-flight copies and MMAs are drained, the TMEM is released and the kernel
 // returns (no trap, no endless loop).
+#include <algorithm>
 #include <atomic>
+#include <cmath>
 #include "common.cuh"
 
 #include <cuda.h>
@@ -117,7 +119,11 @@ struct TcParams {
     float* hf;
     __nv_bfloat16* y;
     int* status;
-    int T, H, G, nblk;
+    int T, H, G;
+    int tseg, nseg;              // tokens per segment (a multiple of kBlk) and segments per sequence
+    float* seg_state;            // [b][H][nseg-1][P][N] fp32: a segment's local end state, then
+                                 // (after the scan) the state entering the next segment
+    float* seg_logdecay;         // [b][H][nseg-1]: sum of dt*A over a segment
     unsigned long long wait_ns;  // limit of every bounded wait
     int starve;                  // failure-detection test: the producer issues no loads
 };
@@ -335,9 +341,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int hd = blockIdx.x, bi = blockIdx.y;
-    const int T = prm.T, H = prm.H, nblk = prm.nblk;
+    const int hd = blockIdx.x, bi = blockIdx.y, seg = blockIdx.z;
+    const int T = prm.T, H = prm.H;
     const int g = hd / (H / prm.G);
+    // this CTA's tokens: [tb, tb + tseg) clipped to T, in blocks of kBlk
+    const int tb = seg * prm.tseg;
+    const int nblk = (min(prm.tseg, T - tb) + kBlk - 1) / kBlk;
 
     uint8_t* small = smem + kSmall;
     uint64_t* bars = reinterpret_cast<uint64_t*>(small);              // BAR_COUNT barriers
@@ -384,7 +393,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             int issued = 0;
             for (int u = 0; u < nblk; ++u) {
                 const int s2 = u & 1, s3 = u % 3;
-                const int t0 = u * kBlk;
+                const int t0 = tb + u * kBlk;
                 if (u >= 2 && !mbar_wait(bar(BAR_EMPTYCB + s2), ((u - 2) >> 1) & 1, s_abort, prm.status, 1)) break;
                 const uint32_t fcb = bar(BAR_FULLCB + s2);
                 const uint32_t slot = sbase + s2 * kCBSlot;
@@ -622,11 +631,16 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         const int r = q * 32 + lane;  // token row (w o X, y) and state row n (S, H)
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
         const float Ah = prm.A[hd];
-        const size_t hbase = ((size_t)bi * H + hd) * kP * kN;
         const int p0 = half * 32;  // this warp's 32 of the 64 p columns
         float Hs[32];              // fp32 running state H[p0 + k][r]
+        {
+            // state entering the segment: h0 for the first, the scanned segment states after it
+            const float* h0 = seg > 0 ? prm.seg_state + (((size_t)bi * H + hd) * (prm.nseg - 1) + seg - 1) * kP * kN
+                              : prm.h0 ? prm.h0 + ((size_t)bi * H + hd) * kP * kN
+                                       : nullptr;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) Hs[k] = prm.h0 ? prm.h0[hbase + (size_t)(p0 + k) * kN + r] : 0.f;
+            for (int k = 0; k < 32; ++k) Hs[k] = h0 ? h0[(size_t)(p0 + k) * kN + r] : 0.f;
+        }
         auto write_sh = [&]() {  // bf16 H^T row r, chunks [4 half, 4 half + 4)
             uint8_t* dst = smem + kSH;
 #pragma unroll
@@ -645,7 +659,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         bool live = __all_sync(0xffffffffu, !*s_abort);
         bool stopped = false;
         auto load_dt = [&](int u) {
-            const int tok = u * kBlk + r;
+            const int tok = tb + u * kBlk + r;
             return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;
         };
         // dt is fetched two blocks ahead: under full HBM load its latency is microseconds
@@ -719,9 +733,10 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             }
             cs_last_prev = cs_last;
         }
-        if (!stopped && live && !*s_abort && prm.hf) {
+        if (!stopped && live && !*s_abort && prm.hf && seg == prm.nseg - 1) {
+            float* hf = prm.hf + ((size_t)bi * H + hd) * kP * kN;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) prm.hf[hbase + (size_t)(p0 + j) * kN + r] = Hs[j];
+            for (int j = 0; j < 32; ++j) hf[(size_t)(p0 + j) * kN + r] = Hs[j];
         }
     } else {
         // ================================================================ y-store warp
@@ -733,7 +748,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             for (int k = 0; k < nblk; ++k) {
                 const int s3 = k % 3;
                 if (!mbar_wait(bar(BAR_YSTAGED + s3), (k / 3) & 1, s_abort, prm.status, 20)) break;
-                tma_store_4d(sbase + kXRing + s3 * kRegion, &prm.tm_y, 0, hd, k * kBlk, bi);
+                tma_store_4d(sbase + kXRing + s3 * kRegion, &prm.tm_y, 0, hd, tb + k * kBlk, bi);
                 bulk_commit();
                 bulk_wait_read0();
                 mbar_arrive(bar(BAR_EMPTYX + s3));
@@ -751,6 +766,232 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+// ------------------------------------------------------------------ segment state pass
+// For a sequence split into segments, the state a segment leaves behind when it starts
+// from zero ("Chunked recurrence" run over the segment alone): H_loc = sum over its blocks
+// of the decayed block states B^T (w o X), and the segment's total log decay sum(dt*A).
+// A scan over segments then gives every segment its entering state.  Only the state
+// recurrence runs here: one CTA per (head, sequence, segment), two CTAs per SM.
+//
+//   warp 0       TMA producer: B (two 64-column boxes) and X of a block into ring slot
+//                u & 1, two blocks ahead
+//   warp 1       TMEM owner and MMA issuer: S(u)^T = B^T (w o X) into TMEM buffer u & 1;
+//                its completion frees the slot
+//   warps 2-9    state group: block prefix sums, w o X in place over X in the slot,
+//                H <- exp(cs_last) H + S in registers
+constexpr int kSThreads = 64 + kGroupThreads;
+constexpr uint32_t kSSlot = 3 * kRegion;             // B (n 0..63, 64..127), then X
+constexpr uint32_t kSX = 2 * kRegion;
+constexpr uint32_t kSSmall = 2 * kSSlot;
+constexpr uint32_t kSSmemBytes = kSSmall + 1024;
+constexpr uint32_t kSTmemCols = 128;                 // two 64-column S buffers
+enum { SB_FULL = 0, SB_EMPTY = 2, SB_XS = 4, SB_ACC = 6, SB_SFREE = 8, SB_DONE = 10, SB_COUNT };
+
+__global__ void __launch_bounds__(kSThreads, 2)
+ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hd = blockIdx.x, bi = blockIdx.y, seg = blockIdx.z;
+    const int T = prm.T, H = prm.H;
+    const int g = hd / (H / prm.G);
+    const int tb = seg * prm.tseg;
+    const int nblk = (min(prm.tseg, T - tb) + kBlk - 1) / kBlk;
+
+    uint8_t* small = smem + kSSmall;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(small);
+    float* s_tot = reinterpret_cast<float*>(small + 128);          // [2][4] quadrant sums
+    volatile int* s_abort = reinterpret_cast<volatile int*>(small + 192);
+    volatile int* s_ystop = s_abort + 1;                           // [2]
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(small + 208);
+    const uint32_t sbase = smem_u32(smem);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+    if (threadIdx.x == 0) {
+        const bool misaligned = (sbase & 1023u) != 0;
+        if (misaligned) atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (2 << 8));
+        for (int i = 0; i < SB_COUNT; ++i)
+            mbar_init(bar(i), (i == SB_XS || i == SB_XS + 1 || i == SB_SFREE || i == SB_SFREE + 1) ? kGroupThreads : 1);
+        *s_abort = misaligned ? 1 : 0;
+        s_wait_ns = prm.wait_ns;
+        s_ystop[0] = s_ystop[1] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
+                     "r"(kSTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == 0) {
+        // ================================================================ TMA producer
+        if (lane == 0 && !*s_abort && !prm.starve) {
+            int issued = 0;
+            for (int u = 0; u < nblk; ++u) {
+                // slot u & 1 is free once S(u-2) has read it
+                if (u >= 2 && !mbar_wait(bar(SB_EMPTY + (u & 1)), ((u - 2) >> 1) & 1, s_abort, prm.status, 40)) break;
+                const uint32_t f = bar(SB_FULL + (u & 1));
+                const uint32_t slot = sbase + (u & 1) * kSSlot;
+                const int t0 = tb + u * kBlk;
+                mbar_expect_tx(f, 3 * kRegion);
+                tma_load_4d(slot, &prm.tm_B, f, 0, g, t0, bi);
+                tma_load_4d(slot + kRegion, &prm.tm_B, f, 64, g, t0, bi);
+                tma_load_4d(slot + kSX, &prm.tm_x, f, 0, hd, t0, bi);
+                issued = u + 1;
+            }
+            for (int u = issued - 2; u < issued; ++u)
+                if (u >= 0) mbar_drain(bar(SB_FULL + (u & 1)), (u >> 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ================================================================ MMA issuer
+        constexpr uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // A B^T (MN-major), B w o X (MN-major)
+        auto wt = [&](int b, uint32_t parity, int where) {
+            return warp_wait(bar(b), parity, s_abort, prm.status, where);
+        };
+        bool ok = __all_sync(0xffffffffu, !*s_abort);
+        if (ok) {
+            for (int u = 0; u < nblk && ok; ++u) {
+                // S buffer u & 1 was last read by the state group for block u - 2
+                ok = wt(SB_FULL + (u & 1), (u >> 1) & 1, 41) && wt(SB_XS + (u & 1), (u >> 1) & 1, 42) &&
+                     (u < 2 || wt(SB_SFREE + (u & 1), ((u - 2) >> 1) & 1, 43));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t slot = sbase + (u & 1) * kSSlot;
+                const uint64_t dBt = sdesc(slot, kRegion, 1024), dXs = sdesc(slot + kSX, kRegion, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kBlk / 16; ++kk)
+                    mma_ss_w(tmem + (u & 1) * 64, dBt + kk * 128, dXs + kk * 128, id_s, kk > 0);
+                mma_commit_w(bar(SB_ACC + (u & 1)));
+                mma_commit_w(bar(SB_EMPTY + (u & 1)));
+            }
+            mma_commit_w(bar(SB_DONE));
+            mbar_drain(bar(SB_DONE), 0);
+        }
+    } else {
+        // ================================================================ state group
+        const int q = warp & 3, half = (warp - 2) >> 2;
+        const int r = q * 32 + lane;  // token row of a block (w o X) and state row n (S, H)
+        const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+        const int p0 = half * 32;
+        const float Ah = prm.A[hd];
+        float Hs[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) Hs[k] = 0.f;
+        auto load_dt = [&](int u) {
+            const int tok = tb + u * kBlk + r;
+            return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;
+        };
+        bool live = __all_sync(0xffffffffu, !*s_abort);
+        bool stopped = false;
+        float dt_a = load_dt(0), dt_b = load_dt(1);
+        float cs_last_prev = 0.f, logsum = 0.f;
+        // iteration u: w o X of block u, then the state update with S(u-1)
+        for (int u = 0; u <= nblk; ++u) {
+            const int s = u & 1;
+            const float dtv = dt_a;
+            dt_a = dt_b;
+            dt_b = load_dt(u + 2);
+            if (!live || *s_abort) s_ystop[s] = 1;
+            float cend[4], cs_last;
+            const float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_tot + s * 4, 4, cs_last, cend);
+            if (s_ystop[s]) {
+                stopped = true;
+                break;
+            }
+            if (live && u < nblk) {
+                live = warp_wait(bar(SB_FULL + s), (u >> 1) & 1, s_abort, prm.status, 44);
+                if (live) {
+                    // w_j x_j in place, one packed bf16x2 multiply per element pair
+                    const __nv_bfloat162 w2 = __float2bfloat162_rn(__expf(cs_last - cs) * dtv);
+                    uint8_t* xs = smem + s * kSSlot + kSX;
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint4 uv = *reinterpret_cast<const uint4*>(xs + swz(r, half * 4 + c4));
+                        __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&uv);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) e[j] = __hmul2(e[j], w2);
+                        *reinterpret_cast<uint4*>(xs + swz(r, half * 4 + c4)) = uv;
+                    }
+                    fence_proxy_async();
+                    mbar_arrive(bar(SB_XS + s));
+                }
+            }
+            if (live && u >= 1) {
+                // H <- exp(cs_last(u-1)) H + S(u-1)
+                const int sp = (u - 1) & 1;
+                live = warp_wait(bar(SB_ACC + sp), ((u - 1) >> 1) & 1, s_abort, prm.status, 45);
+                if (live) {
+                    tc_fence_after();
+                    uint32_t raw[32];
+                    SSD_TMEM_LD32(tmem + lane_addr + sp * 64 + p0, raw);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(bar(SB_SFREE + sp));
+                    const float gam = __expf(cs_last_prev);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) Hs[j] = fmaf(gam, Hs[j], __uint_as_float(raw[j]));
+                }
+            }
+            cs_last_prev = cs_last;
+            if (u < nblk) logsum += cs_last;
+        }
+        if (!stopped && live && !*s_abort) {
+            const size_t o = ((size_t)bi * H + hd) * (prm.nseg - 1) + seg;
+            float* dst = prm.seg_state + o * kP * kN;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dst[(size_t)(p0 + j) * kN + r] = Hs[j];
+            if (r == 0 && half == 0) prm.seg_logdecay[o] = logsum;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kSTmemCols));
+    }
+}
+
+// Entering state of every segment after the first, in place of the local states:
+// H_in(s + 1) = exp(logdecay(s)) H_in(s) + H_loc(s), H_in(0) = h0.  Each (sequence,
+// head) state is spread over kScanSplit CTAs; a thread carries kScanPer entries through
+// the segments, loading kScanBatch segments' worth before the dependent updates.
+constexpr int kScanSplit = 8, kScanThreads = 128, kScanPer = kP * kN / (kScanSplit * kScanThreads), kScanBatch = 4;
+__global__ void __launch_bounds__(kScanThreads) ssd_segment_scan_kernel(const float* h0, float* seg_state,
+                                                                         const float* seg_logdecay, int H, int nseg) {
+    const int hd = blockIdx.x, bi = blockIdx.y;
+    const size_t o = ((size_t)bi * H + hd) * (nseg - 1);
+    const int e0 = blockIdx.z * (kP * kN / kScanSplit) + threadIdx.x;  // entries e0 + kScanThreads * k
+    const float* h0p = h0 ? h0 + ((size_t)bi * H + hd) * kP * kN : nullptr;
+    float run[kScanPer];
+#pragma unroll
+    for (int k = 0; k < kScanPer; ++k) run[k] = h0p ? h0p[e0 + kScanThreads * k] : 0.f;
+    for (int s0 = 0; s0 + 1 < nseg; s0 += kScanBatch) {
+        float v[kScanBatch][kScanPer], gam[kScanBatch];
+#pragma unroll
+        for (int j = 0; j < kScanBatch; ++j) {
+            const bool in = s0 + j + 1 < nseg;
+            gam[j] = in ? __expf(seg_logdecay[o + s0 + j]) : 0.f;
+            const float* w = seg_state + (o + s0 + j) * kP * kN;
+#pragma unroll
+            for (int k = 0; k < kScanPer; ++k) v[j][k] = in ? w[e0 + kScanThreads * k] : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < kScanBatch; ++j) {
+            if (s0 + j + 1 >= nseg) break;
+            float* w = seg_state + (o + s0 + j) * kP * kN;
+#pragma unroll
+            for (int k = 0; k < kScanPer; ++k) {
+                run[k] = fmaf(gam[j], run[k], v[j][k]);
+                w[e0 + kScanThreads * k] = run[k];
+            }
+        }
     }
 }
 
@@ -785,12 +1026,79 @@ int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_
 
 bool prefill_tc_supported(int P, int N, int io) { return io == SSD_BF16 && P == kP && N == kN; }
 
-size_t prefill_tc_workspace_bytes() { return 256; }
+namespace {
+constexpr size_t kSegOffset = 512;  // status word and launch scratch come first
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+int sm_count() {
+    static int n = 0;
+    if (n <= 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+// Segments per sequence.  One CTA walks a segment's blocks one after another, so the
+// fused pass costs about (blocks per CTA) x (waves of CTAs) block-times when the waves
+// are full and about (all blocks / SMs) when CTAs of a ragged last wave finish early;
+// the model takes the mean of the two; a CTA's start (TMEM allocation, first loads) costs
+// about two more block-times.  Splitting the sequence adds CTAs when b * H alone leaves
+// SMs idle, at the price of the state pass (two CTAs per SM, measured at about 0.7 of a
+// fused block-time per block), the scan (about 0.4 block-times per segment) and a fixed
+// cost for the two extra launches.  nseg = 1 wherever the split does not pay by 5 %.
+constexpr double kStatePassPerBlock = 0.7;
+constexpr double kCtaStartBlocks = 2.0;
+constexpr double kScanPerSegment = 0.4;
+constexpr double kSplitFixedBlocks = 5.0;
+std::atomic<int> g_force_nseg{0};
+void plan_segments(int b, int T, int H, int* nseg, int* tseg) {
+    const int nb = (T + kBlk - 1) / kBlk;
+    if (const int f = g_force_nseg.load()) {
+        const int bps = (nb + std::min(f, nb) - 1) / std::min(f, nb);
+        *tseg = bps * kBlk;
+        *nseg = (nb + bps - 1) / bps;
+        return;
+    }
+    const double sms = sm_count();
+    const double units = (double)b * H;
+    double best = 0.0;
+    int best_bps = nb;
+    for (int bps = nb; bps >= 1; --bps) {
+        const int n = (nb + bps - 1) / bps;
+        if (bps < nb && (nb + bps) / (bps + 1) == n) continue;  // same segment count as a longer bps
+        const double len = bps + kCtaStartBlocks;
+        const double waves = std::ceil(units * n / sms) * len;
+        const double flow = std::max(units * n * len / sms, len);
+        double cost = 0.5 * (waves + flow);
+        if (n > 1)
+            cost += kStatePassPerBlock * std::ceil(units * (n - 1) / (2.0 * sms)) * len + kScanPerSegment * n +
+                    kSplitFixedBlocks;
+        if (bps == nb || cost < 0.95 * best) {
+            best = cost;
+            best_bps = bps;
+        }
+    }
+    *tseg = best_bps * kBlk;
+    *nseg = (nb + best_bps - 1) / best_bps;
+}
+}  // namespace
+
+size_t prefill_tc_workspace_bytes(int b, int T, int H) {
+    int nseg = 1, tseg = T;
+    plan_segments(b, T, H, &nseg, &tseg);
+    if (nseg == 1) return kSegOffset;
+    const size_t units = (size_t)b * H * (nseg - 1);
+    return kSegOffset + align256(units * kP * kN * sizeof(float)) + align256(units * sizeof(float));
+}
 
 namespace {
 std::atomic<unsigned long long> g_starve_ns{0};
 }
 void prefill_tc_starve_next(unsigned long long wait_ns) { g_starve_ns.store(wait_ns); }
+void prefill_tc_force_segments(int nseg) { g_force_nseg.store(nseg); }
 
 int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt, const float* A, const void* Bm,
                       const void* Cm, const float* D, const float* h0, void* y, float* hf, void* ws,
@@ -812,16 +1120,36 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     prm.T = T;
     prm.H = H;
     prm.G = G;
-    prm.nblk = (T + kBlk - 1) / kBlk;
+    plan_segments(b, T, H, &prm.nseg, &prm.tseg);
+    const size_t units = (size_t)b * H * (prm.nseg - 1);
+    prm.seg_state = reinterpret_cast<float*>(static_cast<char*>(ws) + kSegOffset);
+    prm.seg_logdecay = reinterpret_cast<float*>(static_cast<char*>(ws) + kSegOffset +
+                                                align256(units * kP * kN * sizeof(float)));
     const unsigned long long starve_ns = g_starve_ns.exchange(0);
     prm.starve = starve_ns != 0;
     prm.wait_ns = starve_ns ? starve_ns : kWaitLimitNs;
     SSD_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), s));
+    if (prm.nseg > 1) {
+        // local end states of all segments but the last, then their scan
+        SSD_CUDA_TRY(cudaFuncSetAttribute(ssd_segment_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)kSSmemBytes));
+        {
+            LaunchScope ls("ssd_segment_state", s);
+            ssd_segment_state_kernel<<<dim3(H, b, prm.nseg - 1), kSThreads, kSSmemBytes, s>>>(prm);
+        }
+        SSD_CUDA_TRY(cudaGetLastError());
+        {
+            LaunchScope ls("ssd_segment_scan", s);
+            ssd_segment_scan_kernel<<<dim3(H, b, kScanSplit), kScanThreads, 0, s>>>(h0, prm.seg_state, prm.seg_logdecay,
+                                                                                    H, prm.nseg);
+        }
+        SSD_CUDA_TRY(cudaGetLastError());
+    }
     SSD_CUDA_TRY(cudaFuncSetAttribute(ssd_prefill_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kSmemBytes));
     {
         LaunchScope ls("ssd_prefill_fused", s);
-        ssd_prefill_fused_kernel<<<dim3(H, b), kThreads, kSmemBytes, s>>>(prm);
+        ssd_prefill_fused_kernel<<<dim3(H, b, prm.nseg), kThreads, kSmemBytes, s>>>(prm);
     }
     SSD_CUDA_TRY(cudaGetLastError());
     return SSD_OK;

@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill_check.restype = _i
         L.ssd_debug_starve_next_prefill.argtypes = [ctypes.c_ulonglong]
         L.ssd_debug_starve_next_prefill.restype = _i
+        L.ssd_debug_force_prefill_segments.argtypes = [_i]
+        L.ssd_debug_force_prefill_segments.restype = _i
         L.ssd_decode_workspace_size.argtypes = [_i] * 3
         L.ssd_decode_workspace_size.restype = _sz
         L.ssd_decode_step.argtypes = [_i] * 9 + [_vp] * 10 + [_sz, _vp]
@@ -190,6 +192,12 @@ def debug_starve_next_prefill(wait_limit_s=0.1):
     """Failure-detection test hook: the next tensor-core prefill issues no loads, so its
     bounded waits expire after `wait_limit_s` and prefill_check raises SSD_ERR_TIMEOUT."""
     _check(lib().ssd_debug_starve_next_prefill(int(wait_limit_s * 1e9)), "ssd_debug_starve_next_prefill")
+
+
+def debug_force_prefill_segments(nseg=0):
+    """Test hook: split every following tensor-core prefill into `nseg` sequence segments
+    (0 = let the cost model choose)."""
+    _check(lib().ssd_debug_force_prefill_segments(int(nseg)), "ssd_debug_force_prefill_segments")
 
 
 def decode_workspace_size(layers, b, G) -> int:

@@ -158,6 +158,23 @@ def test_binding_refuses_cpu_tensors():
                     torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16), torch.zeros(4))
 
 
+def test_segment_hook_and_workspace():
+    """The split of a sequence into segments sizes the workspace: one fp32 state and one
+    log decay per (sequence, head) for every segment but the last."""
+    args = (1, 4096, 24, 64, 128, 1, 256, 1)
+    assert ssd.lib().ssd_debug_force_prefill_segments(-1) == 1  # SSD_ERR_INVALID_ARG
+    try:
+        ssd.debug_force_prefill_segments(1)
+        one = ssd.prefill_workspace_size(*args)
+        ssd.debug_force_prefill_segments(4)
+        four = ssd.prefill_workspace_size(*args)
+        assert four - one >= 3 * 24 * (64 * 128 * 4 + 4)
+        ssd.debug_force_prefill_segments(1000)  # clamped to one block per segment
+        assert ssd.prefill_workspace_size(*args) - one >= 31 * 24 * 64 * 128 * 4
+    finally:
+        ssd.debug_force_prefill_segments(0)
+
+
 def test_starve_hook_rejects_out_of_range_limits():
     import state_space_model_04_b200 as ssd
     L = ssd.lib()

@@ -84,13 +84,20 @@ def test_long_context_sampled(L):
 
 
 def test_fused_kernel_is_the_bf16_path():
-    """bf16 with P=64, N=128 runs the single fused tensor-core kernel; other shapes and fp32
-    run the four-kernel path."""
-    case = make_prefill(1, 512, 4, 64, 128, 1, 256, "bf16", seed=15)
+    """bf16 with P=64, N=128 runs the fused tensor-core kernel, preceded by the segment state
+    pass and scan when the sequences are split (few sequence-heads for the SMs); other
+    shapes and fp32 run the four-kernel path."""
+    case = make_prefill(8, 512, 80, 64, 128, 1, 256, "bf16", seed=15)
     ssd.profile_begin()
     run_prefill(ssd, case)
     kt = ssd.profile_end()
     assert list(kt) == ["ssd_prefill_fused"] and kt["ssd_prefill_fused"][0] == 1
+    case = make_prefill(1, 4096, 24, 64, 128, 1, 256, "bf16", seed=15)  # the 130M-layer shape splits
+    ssd.profile_begin()
+    run_prefill(ssd, case)
+    kt = ssd.profile_end()
+    assert {k: v[0] for k, v in kt.items()} == {"ssd_segment_state": 1, "ssd_segment_scan": 1,
+                                                 "ssd_prefill_fused": 1}
     case = make_prefill(1, 512, 4, 64, 64, 1, 256, "bf16", seed=15)
     ssd.profile_begin()
     run_prefill(ssd, case)
@@ -106,13 +113,41 @@ def test_deterministic_bitwise():
     assert torch.equal(y1, y2) and torch.equal(h1, h2)
 
 
-def test_batch_invariance_bitwise():
+@pytest.mark.parametrize("nseg", [1, 3])
+def test_batch_invariance_bitwise(nseg):
+    """A sequence's result does not depend on the rest of the batch, bit for bit, for a
+    given split of the sequences into segments (the automatic split depends on b * H)."""
     case = make_prefill(3, 520, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=6)
-    y, hf, t = run_prefill(ssd, case)
-    y1, h1 = ssd.prefill(t["x"][1:2].contiguous(), t["dt"][1:2].contiguous(), t["A"], t["B"][1:2].contiguous(),
-                         t["C"][1:2].contiguous(), t["D"], chunk=256, h0=t["h0"][1:2].contiguous())
-    torch.cuda.synchronize()
+    ssd.debug_force_prefill_segments(nseg)
+    try:
+        y, hf, t = run_prefill(ssd, case)
+        y1, h1 = ssd.prefill(t["x"][1:2].contiguous(), t["dt"][1:2].contiguous(), t["A"], t["B"][1:2].contiguous(),
+                             t["C"][1:2].contiguous(), t["D"], chunk=256, h0=t["h0"][1:2].contiguous())
+        torch.cuda.synchronize()
+    finally:
+        ssd.debug_force_prefill_segments(0)
     assert torch.equal(y[1:2], y1) and torch.equal(hf[1:2], h1)
+
+
+@pytest.mark.parametrize("nseg", [1, 2, 3, 8])
+def test_sequence_split_matches_oracle(nseg):
+    """Splitting each sequence into segments (local end states, a scan over them, then the
+    fused pass from each segment's entering state) is the same function as one pass:
+    within the bf16 bound of the oracle, and close to the unsplit result.  T = 1000 leaves
+    a ragged last segment; grouped B/C and a non-zero h0."""
+    case = make_prefill(2, 1000, 6, 64, 128, 3, 256, "bf16", h0_std=0.1, seed=21)
+    ssd.debug_force_prefill_segments(1)
+    try:
+        y1, h1, _ = run_prefill(ssd, case)
+        ssd.debug_force_prefill_segments(nseg)
+        y, hf, _ = run_prefill(ssd, case)
+    finally:
+        ssd.debug_force_prefill_segments(0)
+    y_ref, hf_ref = oracle_subset(case, range(case.b), range(case.H))
+    check(_np(y), y_ref, "bf16", "y")
+    check(_np(hf), hf_ref, "bf16", "h_final")
+    check(_np(y), _np(y1), "bf16", "y split vs one pass")
+    check(_np(hf), _np(h1), "bf16", "h_final split vs one pass")
 
 
 def test_causality_bitwise():
