@@ -296,6 +296,10 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024, help="timed decode steps at batch 1")
     ap.add_argument("--decode-batches", default="1,32")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-loop-compare", action="store_true",
+                    help="skip the decode loop and recompute comparisons")
+    ap.add_argument("--skip-other-prefill", action="store_true",
+                    help="skip the 130M-layer and long-context prefill timings")
     ap.add_argument("--prefill-batch", type=int, default=PB,
                     help="sequences per prefill step (default: the 2.7B-layer configuration's 8); "
                          "smaller values are for profiling captures only")
@@ -455,6 +459,13 @@ def main():
                                           max_over_ranks, world, pk, box)
         launches += box[0]
 
+    # ---------------- the other prefill configurations
+    other = {}
+    if not args.skip_other_prefill:
+        box = [0]
+        other = bench_prefill_configs(ssd, torch, dev, stream, args, clocks, barrier, max_over_ranks, world, pk, box)
+        launches += box[0]
+
     clk = clocks.stop()
 
     cpu = None
@@ -474,10 +485,67 @@ def main():
                 "hbm_gbs_alg": pbytes * world / (ms * 1e-3) / 1e9,
                 "tensor_frac": tflops / world / pk["bf16_tflops"],
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
-                "clocks": clk, "decode": decode}
+                "clocks": clk, "decode": decode, "prefill_configs": other}
         print(json.dumps(line), flush=True)
     ranks.close()
     return 0
+
+
+def bench_prefill_configs(ssd, torch, dev, stream, args, clocks, barrier, max_over_ranks, world, pk, box):
+    """The other bf16 prefill configurations: the 130M-layer shape (b=1, T=4096, H=24) and
+    the long-context shape (b=1, T=65536, H=80, G=8), timed like the headline (inputs
+    resident, CUDA events on the launching stream, max over ranks).  On the fused path the
+    executed decomposition is the same for every requested chunk length, so one timing
+    serves L = 64, 128 and 256; TFLOP/s is given at each requested L and at the executed
+    128.  Both have few (sequence, head) pairs for 148 SMs, so the sequences are split into
+    segments (state pass + scan + fused pass); the segment count is reported."""
+    from ssd_inputs import make_config
+    out = {}
+    for name, label in (("mamba2_130m_layer", "mamba2_130m_layer"), ("long_context_L256", "long_context")):
+        c = make_config(name)
+        b, T, H, P, N, G = c.b, c.T, c.H, c.P, c.N, c.G
+        def bf(bits):
+            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        x, Bm, Cm = bf(c.x_bits), bf(c.B_bits), bf(c.C_bits)
+        dt, A, D = (torch.from_numpy(v).to(dev) for v in (c.dt, c.A, c.D))
+        y = torch.empty_like(x)
+        hfin = torch.empty(b, H, P, N, device=dev)
+        ws = torch.empty(ssd.prefill_workspace_size(b, T, H, P, N, G, 256, ssd.SSD_BF16), dtype=torch.uint8,
+                         device=dev)
+        def step():
+            ssd.prefill(x, dt, A, Bm, Cm, D, chunk=256, y=y, h_final=hfin, workspace=ws)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        barrier()
+        n_steps = max(3, min(args.steps, 10))
+        n0 = ssd.launch_count()
+        ssd.profile_begin()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0 = time.time()
+        e0.record(stream)
+        for _ in range(n_steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clocks.mark(w0, time.time())
+        kt = ssd.profile_end()
+        box[0] += ssd.launch_count() - n0
+        barrier()
+        ms = max_over_ranks(e0.elapsed_time(e1) / n_steps)
+        byt = prefill_bytes(b, T, H, P, N, G, with_h0=False)
+        gbs = byt * world / (ms * 1e-3) / 1e9
+        entry = {"b": b, "T": T, "H": H, "G": G, "ms_per_step": ms, "tokens_per_s": job_rate(b * T, world, ms),
+                 "bytes_per_step": byt, "hbm_gbs_alg": gbs, "hbm_frac": gbs / world / pk["hbm_gbs"],
+                 "tflops_executed_L128": job_rate(prefill_flops(b, T, H, P, N, G, EXEC_L_FUSED), world, ms) / 1e12,
+                 "tflops_at_requested_L": {str(L): job_rate(prefill_flops(b, T, H, P, N, G, L), world, ms) / 1e12
+                                           for L in ((64, 128, 256) if label == "long_context" else (256,))},
+                 "kernels": {k: {"launches": v[0] // n_steps, "avg_ms": v[1] / max(v[0], 1)} for k, v in kt.items()},
+                 "segments": ssd.prefill_segments(b, T, H, P, N, G, 256, ssd.SSD_BF16)}
+        out[label] = entry
+        del x, Bm, Cm, dt, A, D, y, hfin, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 def bench_decode(ssd, torch, dev, stream, case, hf, b, args, clocks, barrier, max_over_ranks, world, pk, box):
@@ -521,6 +589,10 @@ def bench_decode(ssd, torch, dev, stream, case, hf, b, args, clocks, barrier, ma
     sps = job_rate(steps, world, ms)
     byt = decode_bytes_per_step(DL, b, DH, DP, DN, DG)
     gbs = byt * sps / 1e9
+    loops = {}
+    if b == 1 and not args.skip_loop_compare:
+        loops = bench_decode_loops(ssd, torch, dev, stream, h, cst, xbc, dt, A, D, conv_w, conv_b, ring,
+                                   ms / steps, barrier, max_over_ranks, box)
     ok = bool(torch.isfinite(h).all().item())
     plan.close()
     del h, cst, xbc, dt
@@ -528,7 +600,77 @@ def bench_decode(ssd, torch, dev, stream, case, hf, b, args, clocks, barrier, ma
     return {"batch": b, "layers": DL, "steps": steps, "steps_per_launch": steps_per_launch,
             "steps_per_s": sps, "tokens_per_s": sps * b, "ms_per_step": ms / steps,
             "bytes_per_step": byt, "hbm_gbs_alg": gbs, "hbm_frac": gbs / world / pk["hbm_gbs"],
-            "kernel": "decode_step (graph of %d steps)" % steps_per_launch, "state_finite": ok}
+            "kernel": "decode_step (graph of %d steps)" % steps_per_launch, "state_finite": ok,
+            "loop_compare": loops}
+
+
+def bench_decode_loops(ssd, torch, dev, stream, h, cst, xbc, dt, A, D, conv_w, conv_b, ring, graph_ms_per_step,
+                       barrier, max_over_ranks, box):
+    """The comparisons the pages make for the cached decode, on our kernels at batch 1 and
+    the 2.7B-shaped 64-layer cache ([CF-SSD] O(1) caching and compiled-loop sections):
+      * the on-device loop (one CUDA graph of many steps) against the same steps launched one
+        call at a time, and against a host loop that waits for each step before the next
+        (the host round trip per token a non-compiled loop pays);
+      * the cached step against recomputing the whole 4096-token context: one prefill of
+        b = 1, T = 4096 over the 80 heads, times 64 layers, per generated token.
+    All timed with CUDA events on the launching stream."""
+    n = 128
+    y = torch.empty(DL, 1, DH, DP, dtype=xbc.dtype, device=dev)
+    ws = torch.empty(ssd.decode_workspace_size(DL, 1, DG), dtype=torch.uint8, device=dev)
+
+    def step(t):
+        ssd.decode_step(h, cst, xbc[t % ring], dt[t % ring], A, D, conv_w, conv_b, G=DG, y=y, workspace=ws)
+
+    for t in range(8):
+        step(t)
+    torch.cuda.synchronize()
+    barrier()
+    res = {}
+    for mode in ("launch_per_step", "host_sync_per_step"):
+        n0 = ssd.launch_count()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        for t in range(n):
+            step(t)
+            if mode == "host_sync_per_step":
+                torch.cuda.synchronize()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        box[0] += ssd.launch_count() - n0
+        barrier()
+        res[mode] = max_over_ranks(ev[0].elapsed_time(ev[1])) / n
+    # recompute: prefill of the full context for one sequence, all heads, one layer; x64 layers
+    from ssd_inputs import make_config
+    c = make_config("mamba2_2p7b_layer", b=1, seed=11)
+    def bf(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    px, pB, pC = bf(c.x_bits), bf(c.B_bits), bf(c.C_bits)
+    pdt, pA, pD = (torch.from_numpy(v).to(dev) for v in (c.dt, c.A, c.D))
+    py = torch.empty_like(px)
+    pws = torch.empty(ssd.prefill_workspace_size(1, c.T, c.H, c.P, c.N, c.G, 256, ssd.SSD_BF16), dtype=torch.uint8,
+                      device=dev)
+    for _ in range(3):
+        ssd.prefill(px, pdt, pA, pB, pC, pD, chunk=256, y=py, workspace=pws)
+    torch.cuda.synchronize()
+    barrier()
+    n0 = ssd.launch_count()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    for _ in range(10):
+        ssd.prefill(px, pdt, pA, pB, pC, pD, chunk=256, y=py, workspace=pws)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    box[0] += ssd.launch_count() - n0
+    barrier()
+    prefill_ms = max_over_ranks(ev[0].elapsed_time(ev[1])) / 10
+    recompute_ms = prefill_ms * DL
+    return {"steps": n, "graph_ms_per_step": graph_ms_per_step,
+            "launch_per_step_ms": res["launch_per_step"], "host_sync_per_step_ms": res["host_sync_per_step"],
+            "graph_vs_host_sync": res["host_sync_per_step"] / graph_ms_per_step,
+            "graph_vs_launch_per_step": res["launch_per_step"] / graph_ms_per_step,
+            "recompute_context": c.T, "recompute_prefill_ms_per_layer": prefill_ms,
+            "recompute_ms_per_token": recompute_ms,
+            "cached_vs_recompute_speedup": recompute_ms / graph_ms_per_step}
 
 
 if __name__ == "__main__":

@@ -131,6 +131,13 @@ SSD_API int ssd_debug_starve_next_prefill(unsigned long long wait_limit_ns);
  * Errors: SSD_ERR_INVALID_ARG if nseg < 0. */
 SSD_API int ssd_debug_force_prefill_segments(int nseg);
 
+/* Segments per sequence that ssd_prefill would use for this shape: 1 when the whole
+ * sequence runs in one pass (every shape outside the tensor-core path, and tensor-core
+ * shapes with enough sequence-heads for the SMs of the current device), else the count of
+ * 128-token-aligned segments (see ssd_prefill: local end states, a scan, then the fused
+ * pass per segment).  Returns 0 for an invalid shape.  Host-only; nothing is enqueued. */
+SSD_API int ssd_prefill_segments(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype);
+
 /* ------------------------------------------------------------------------------------
  * Cached decode step  ([CF-SSD] O(1) caching section)
  *

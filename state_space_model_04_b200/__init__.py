@@ -24,6 +24,7 @@ from .ssd import (  # noqa: F401
     profile_end,
     prefill,
     prefill_check,
+    prefill_segments,
     prefill_workspace_size,
     status_string,
 )

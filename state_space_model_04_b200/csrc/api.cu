@@ -28,6 +28,7 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
 int prefill_tc_status(void* ws, cudaStream_t s);
 void prefill_tc_starve_next(unsigned long long wait_ns);
 void prefill_tc_force_segments(int nseg);
+int prefill_tc_segments(int b, int T, int H);
 size_t decode_workspace_bytes(int layers, int b, int G);
 int launch_decode_step(int layers, int b, int H, int N, int G, int act, int io, float* h,
                        float* conv_state, const void* xbc, const float* dt, const float* A,
@@ -212,6 +213,12 @@ int ssd_debug_starve_next_prefill(unsigned long long wait_limit_ns) {
         return set_error(SSD_ERR_INVALID_ARG, "wait_limit_ns %llu outside [1e6, 1e10]", wait_limit_ns);
     prefill_tc_starve_next(wait_limit_ns);
     return SSD_OK;
+}
+
+int ssd_prefill_segments(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype) {
+    if (check_prefill_shape(b, T, H, P, N, G, chunk, io_dtype) != SSD_OK) return 0;
+    if (b == 0 || T == 0 || !prefill_tc_supported(P, N, io_dtype)) return 1;
+    return prefill_tc_segments(b, T, H);
 }
 
 int ssd_debug_force_prefill_segments(int nseg) {

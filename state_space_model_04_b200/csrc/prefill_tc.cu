@@ -1086,6 +1086,12 @@ void plan_segments(int b, int T, int H, int* nseg, int* tseg) {
 }
 }  // namespace
 
+int prefill_tc_segments(int b, int T, int H) {
+    int nseg = 1, tseg = T;
+    plan_segments(b, T, H, &nseg, &tseg);
+    return nseg;
+}
+
 size_t prefill_tc_workspace_bytes(int b, int T, int H) {
     int nseg = 1, tseg = T;
     plan_segments(b, T, H, &nseg, &tseg);

@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill_check.restype = _i
         L.ssd_debug_starve_next_prefill.argtypes = [ctypes.c_ulonglong]
         L.ssd_debug_starve_next_prefill.restype = _i
+        L.ssd_prefill_segments.argtypes = [_i] * 8
+        L.ssd_prefill_segments.restype = _i
         L.ssd_debug_force_prefill_segments.argtypes = [_i]
         L.ssd_debug_force_prefill_segments.restype = _i
         L.ssd_decode_workspace_size.argtypes = [_i] * 3
@@ -192,6 +194,11 @@ def debug_starve_next_prefill(wait_limit_s=0.1):
     """Failure-detection test hook: the next tensor-core prefill issues no loads, so its
     bounded waits expire after `wait_limit_s` and prefill_check raises SSD_ERR_TIMEOUT."""
     _check(lib().ssd_debug_starve_next_prefill(int(wait_limit_s * 1e9)), "ssd_debug_starve_next_prefill")
+
+
+def prefill_segments(b, T, H, P, N, G, chunk, io_dtype) -> int:
+    """Segments per sequence ssd_prefill uses for this shape (1 = one pass; 0 = invalid)."""
+    return int(lib().ssd_prefill_segments(b, T, H, P, N, G, chunk, io_dtype))
 
 
 def debug_force_prefill_segments(nseg=0):

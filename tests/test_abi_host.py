@@ -164,9 +164,15 @@ def test_segment_hook_and_workspace():
     args = (1, 4096, 24, 64, 128, 1, 256, 1)
     assert ssd.lib().ssd_debug_force_prefill_segments(-1) == 1  # SSD_ERR_INVALID_ARG
     try:
+        assert ssd.prefill_segments(*args) >= 1
+        assert ssd.prefill_segments(8, 4096, 80, 64, 128, 1, 256, 1) == 1   # enough sequence-heads
+        assert ssd.prefill_segments(1, 4096, 24, 64, 64, 1, 256, 1) == 1    # N = 64: the SIMT path
+        assert ssd.prefill_segments(1, 512, 4, 64, 64, 1, 100, 0) == 0      # invalid chunk
         ssd.debug_force_prefill_segments(1)
+        assert ssd.prefill_segments(*args) == 1
         one = ssd.prefill_workspace_size(*args)
         ssd.debug_force_prefill_segments(4)
+        assert ssd.prefill_segments(*args) == 4
         four = ssd.prefill_workspace_size(*args)
         assert four - one >= 3 * 24 * (64 * 128 * 4 + 4)
         ssd.debug_force_prefill_segments(1000)  # clamped to one block per segment
