@@ -90,8 +90,10 @@ SSD_API const char* ssd_last_error(void);
  * chunk must be 64, 128 or 256.  x, B, C, dt, A, D must not alias y or h_final.
  * Arithmetic: SSD_BF16 inputs with P == 64 and N == 128 run one fused tensor-core kernel
  * (tcgen05 bf16 contractions, fp32 accumulation, fp32 decay in log space, fp32 running
- * state kept on chip, 128-token blocks); other bf16 shapes and all SSD_F32 inputs run
- * the four-kernel fp32-FMA path with the prefix sums of dt*A kept in fp64 (no TF32).
+ * state kept on chip, 128-token blocks), after a tensor-core state pass and a scan when
+ * few (sequence, head) pairs would leave SMs idle (sequences split into segments, see
+ * ssd_prefill_segments); other bf16 shapes and all SSD_F32 inputs run the four-kernel
+ * fp32-FMA path with the prefix sums of dt*A kept in fp64 (no TF32).
  * The workspace's first 256 bytes hold a device status word (see ssd_prefill_check).
  * Errors: SSD_ERR_INVALID_ARG (null pointer for a required argument, negative size,
  * H % G != 0, bad chunk or dtype, misaligned pointer), SSD_ERR_UNSUPPORTED (P, N),
@@ -104,6 +106,22 @@ SSD_API int ssd_prefill(int b, int T, int H, int P, int N, int G, int chunk, int
                 const void* x, const float* dt, const float* A, const void* B,
                 const void* C, const float* D, const float* h0, void* y, float* h_final,
                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* ssd_prefill from the raw time step: the step size is formed inside the kernels where they
+ * load it ([CF-SSD]: the elementwise chain ahead of the SSD fused into the kernel; the
+ * Mamba-2 block's dt pre-processing), so it never takes a separate pass over memory:
+ *   dt[b][t][h] = min(max(softplus(dt_raw[b][t][h] + dt_bias[h]), dt_min), dt_max),
+ *   softplus(z) = log(1 + exp(z)), computed in fp32 (z itself above 20).
+ *   dt_raw  [b][T][H] fp32      dt_bias [H] fp32, or NULL for no bias
+ *   dt_min, dt_max: 0 <= dt_min < dt_max; dt_max may be +infinity (no upper clamp).
+ * Everything else, the workspace included, is as for ssd_prefill.
+ * Errors: as ssd_prefill, plus SSD_ERR_INVALID_ARG for a clamp range outside the rule above
+ * (NaN included) or a misaligned dt_bias. */
+SSD_API int ssd_prefill_dt_raw(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype,
+                       const void* x, const float* dt_raw, const float* dt_bias, float dt_min,
+                       float dt_max, const float* A, const void* B, const void* C, const float* D,
+                       const float* h0, void* y, float* h_final, void* workspace,
+                       size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream` and returns the device-side status recorded by the most recent
  * ssd_prefill that used `workspace` (SSD_OK, or SSD_ERR_TIMEOUT if a bounded wait inside

@@ -55,6 +55,7 @@ def _load():
         lib.oracle_ssd_quadratic.argtypes = [i] * 6 + [_dp] * 9 + [i]
         lib.oracle_decode_step.argtypes = [i] * 8 + [_dp] * 9 + [i]
         lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_dt_from_raw.argtypes = [ctypes.c_size_t, i, _dp, _dp, ctypes.c_double, ctypes.c_double, _dp]
         _lib = lib
     return _lib
 
@@ -103,6 +104,19 @@ def ssd_chunked(x, dt, A, B, C, D, L, h0=None, nthreads=0):
 def ssd_quadratic(x, dt, A, B, C, D, h0=None, nthreads=0):
     """Whole-sequence quadratic form (one chunk of length T, direct segment sums)."""
     return _prefill(_load().oracle_ssd_quadratic, x, dt, A, B, C, D, h0, None, nthreads)
+
+
+def dt_from_raw(dt_raw, dt_bias=None, dt_min=0.0, dt_max=float("inf")):
+    """Step sizes from the raw projection output: clamp(softplus(dt_raw + dt_bias[h]),
+    dt_min, dt_max) in float64 (the Mamba-2 block's pre-processing of dt, which the paper's
+    compiled graph fuses ahead of the SSD).  dt_raw [..., H]; returns float64 of the same shape."""
+    L = _load()
+    raw = _c(dt_raw)
+    H = raw.shape[-1]
+    bias = None if dt_bias is None else _c(dt_bias)
+    out = np.empty_like(raw)
+    L.oracle_dt_from_raw(raw.size, H, _p(raw), _p(bias), dt_min, dt_max, _p(out))
+    return out
 
 
 def decode_step(h, conv_state, xbc, dt, A, D, conv_w, conv_b, act, G, N, nthreads=0):

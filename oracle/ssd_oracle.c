@@ -299,3 +299,23 @@ void oracle_decode_step(int layers, int b, int H, int P, int N, int G, int kconv
         free(u);
     }
 }
+
+/*
+ * Step sizes from the raw projection output, as the Mamba-2 block forms them before the
+ * SSD ([CF-SSD]: the elementwise chain -- bias add, softplus, clamp -- ahead of the scan,
+ * which the paper fuses into the surrounding computation):
+ *   dt[i] = min(max(softplus(raw[i] + bias[i % H]), lo), hi),  softplus(z) = log(1 + e^z).
+ * The softplus is evaluated as max(z, 0) + log1p(exp(-|z|)), which equals log(1 + e^z)
+ * for every z and never overflows.  bias may be NULL (no bias); hi may be +inf.
+ * n = b * T * H entries in [b][T][H] order.
+ */
+void oracle_dt_from_raw(size_t n, int H, const double* raw, const double* bias, double lo, double hi,
+                        double* dt) {
+    for (size_t i = 0; i < n; ++i) {
+        const double z = raw[i] + (bias ? bias[i % (size_t)H] : 0.0);
+        double sp = (z > 0.0 ? z : 0.0) + log1p(exp(-fabs(z)));
+        if (sp < lo) sp = lo;
+        if (sp > hi) sp = hi;
+        dt[i] = sp;
+    }
+}

@@ -17,12 +17,13 @@ namespace ssd {
 // kernels (defined in the other translation units)
 size_t prefill_simt_workspace_bytes(int b, int T, int H, int N, int L, int io);
 int launch_prefill_simt(int b, int T, int H, int N, int G, int L, int io, const void* x,
-                        const float* dt, const float* A, const void* Bm, const void* Cm,
+                        const float* dt, const DtMap& dtm, const float* A, const void* Bm, const void* Cm,
                         const float* D, const float* h0, void* y, float* hf, void* ws,
                         cudaStream_t s);
 bool prefill_tc_supported(int P, int N, int io);
 size_t prefill_tc_workspace_bytes(int b, int T, int H);
-int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt, const float* A, const void* Bm,
+int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt, const DtMap& dtm, const float* A,
+                      const void* Bm,
                       const void* Cm, const float* D, const float* h0, void* y, float* hf, void* ws,
                       cudaStream_t s);
 int prefill_tc_status(void* ws, cudaStream_t s);
@@ -234,11 +235,10 @@ int ssd_prefill_check(void* workspace, void* stream) {
     return prefill_tc_status(workspace, static_cast<cudaStream_t>(stream));
 }
 
-int ssd_prefill(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype,
-                const void* x, const float* dt, const float* A, const void* B, const void* C,
-                const float* D, const float* h0, void* y, float* h_final, void* workspace,
-                size_t workspace_bytes, void* stream) {
-    g_detail[0] = 0;
+static int prefill_impl(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype, const void* x,
+                        const float* dt, const DtMap& dtm, const float* A, const void* B, const void* C,
+                        const float* D, const float* h0, void* y, float* h_final, void* workspace,
+                        size_t workspace_bytes, void* stream) {
     SSD_CHECK(check_prefill_shape(b, T, H, P, N, G, chunk, io_dtype));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t state_bytes = (size_t)b * H * P * N * sizeof(float);
@@ -281,10 +281,36 @@ int ssd_prefill(int b, int T, int H, int P, int N, int G, int chunk, int io_dtyp
     for (int i = 0; i < 7; ++i)
         if (overlaps({workspace, need}, rin[i])) return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps %s", names[i]);
     if (prefill_tc_supported(P, N, io_dtype))
-        return launch_prefill_tc(b, T, H, G, x, dt, A, B, C, D, h0, y, h_final, workspace, s);
+        return launch_prefill_tc(b, T, H, G, x, dt, dtm, A, B, C, D, h0, y, h_final, workspace, s);
     SSD_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(int), s));
-    return launch_prefill_simt(b, T, H, N, G, chunk, io_dtype, x, dt, A, B, C, D, h0, y, h_final,
+    return launch_prefill_simt(b, T, H, N, G, chunk, io_dtype, x, dt, dtm, A, B, C, D, h0, y, h_final,
                                static_cast<char*>(workspace) + kStatusBytes, s);
+}
+
+int ssd_prefill(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype,
+                const void* x, const float* dt, const float* A, const void* B, const void* C,
+                const float* D, const float* h0, void* y, float* h_final, void* workspace,
+                size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    const DtMap plain{nullptr, 0.f, 0.f, 0};
+    return prefill_impl(b, T, H, P, N, G, chunk, io_dtype, x, dt, plain, A, B, C, D, h0, y, h_final, workspace,
+                        workspace_bytes, stream);
+}
+
+int ssd_prefill_dt_raw(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype,
+                       const void* x, const float* dt_raw, const float* dt_bias, float dt_min, float dt_max,
+                       const float* A, const void* B, const void* C, const float* D, const float* h0,
+                       void* y, float* h_final, void* workspace, size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    if (!(dt_min >= 0.f) || !(dt_max > dt_min))  // also rejects NaN limits
+        return set_error(SSD_ERR_INVALID_ARG, "dt clamp range [%g, %g] must satisfy 0 <= dt_min < dt_max",
+                         (double)dt_min, (double)dt_max);
+    SSD_CHECK(check_ptr(dt_bias, "dt_bias", false));
+    if (dt_bias && H > 0 && overlaps({dt_bias, (size_t)H * 4}, {y, (size_t)b * T * H * P * (io_dtype == SSD_BF16 ? 2 : 4)}))
+        return set_error(SSD_ERR_INVALID_ARG, "y overlaps input dt_bias");
+    const DtMap raw{dt_bias, dt_min, dt_max, 1};
+    return prefill_impl(b, T, H, P, N, G, chunk, io_dtype, x, dt_raw, raw, A, B, C, D, h0, y, h_final, workspace,
+                        workspace_bytes, stream);
 }
 
 size_t ssd_decode_workspace_size(int layers, int b, int G) {

@@ -28,6 +28,25 @@ __device__ __forceinline__ void store_io(__nv_bfloat16* p, size_t i, float v) {
     p[i] = __float2bfloat16_rn(v);
 }
 
+// Time step as the prefill kernels read it.  By default dt arrives already positive (the
+// softplus applied by the caller) and is used as is.  With `raw` set, the kernels apply the
+// pre-processing of the Mamba-2 block where they load it, so the raw projection output
+// never takes a separate pass over memory ("Compiler-First State Space Duality and
+// Portable O(1) Autoregressive Caching": the elementwise chain ahead of the SSD fused into
+// the kernel): dt = clamp(softplus(dt_raw + bias[h]), lo, hi), softplus(z) = log(1 + e^z)
+// (taken as z above 20, where the two differ by less than fp32 rounding).
+struct DtMap {
+    const float* bias;  // [H] or nullptr (zero bias)
+    float lo, hi;       // clamp range (hi may be +inf)
+    int raw;            // 0: dt is used as given
+};
+__device__ __forceinline__ float dt_value(float v, const DtMap& m, int h) {
+    if (!m.raw) return v;
+    const float z = v + (m.bias ? __ldg(m.bias + h) : 0.f);
+    const float sp = z > 20.f ? z : log1pf(expf(z));
+    return fminf(fmaxf(sp, m.lo), m.hi);
+}
+
 // Map a CUDA error to a status with detail.
 int cuda_status(cudaError_t e, const char* where);
 

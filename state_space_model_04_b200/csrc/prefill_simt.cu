@@ -33,7 +33,7 @@ __device__ __forceinline__ float exp_cs(float v) { return expf(v); }
 // ---------------------------------------------------------------- K1
 template <typename CsT>
 __global__ void __launch_bounds__(kThreads)
-decay_cumsum_kernel(int T, int H, int L, int nc, const float* __restrict__ dt,
+decay_cumsum_kernel(int T, int H, int L, int nc, const float* __restrict__ dt, const DtMap dtm,
                     const float* __restrict__ A, CsT* __restrict__ cs) {
     const int c = blockIdx.x, hd = blockIdx.y, bi = blockIdx.z;
     const int t0 = c * L, Lc = min(L, T - t0);
@@ -45,7 +45,7 @@ decay_cumsum_kernel(int T, int H, int L, int nc, const float* __restrict__ dt,
     for (int base = 0; base < L; base += kThreads) {
         const int j = base + threadIdx.x;
         CsT v = CsT(0);
-        if (j < Lc) v = (CsT)dt[((size_t)bi * T + t0 + j) * H + hd] * a_h;
+        if (j < Lc) v = (CsT)dt_value(dt[((size_t)bi * T + t0 + j) * H + hd], dtm, hd) * a_h;
         // warp inclusive scan
         const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
@@ -69,7 +69,7 @@ decay_cumsum_kernel(int T, int H, int L, int nc, const float* __restrict__ dt,
 template <typename IoT, typename CsT, int N>
 __global__ void __launch_bounds__(kThreads)
 chunk_state_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ x,
-                   const float* __restrict__ dt, const IoT* __restrict__ Bm,
+                   const float* __restrict__ dt, const DtMap dtm, const IoT* __restrict__ Bm,
                    const CsT* __restrict__ cs, float* __restrict__ S) {
     constexpr int KT = 32;                 // tokens per smem stage
     constexpr int NT = N / 8;              // thread columns (8 n each)
@@ -94,7 +94,7 @@ chunk_state_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ x
     for (int k0 = 0; k0 < Lc; k0 += KT) {
         if (threadIdx.x < KT) {
             const int t = k0 + threadIdx.x;
-            sW[threadIdx.x] = t < Lc ? exp_cs(cs_last - csc[t]) * dt[((size_t)bi * T + t0 + t) * H + hd] : 0.f;
+            sW[threadIdx.x] = t < Lc ? exp_cs(cs_last - csc[t]) * dt_value(dt[((size_t)bi * T + t0 + t) * H + hd], dtm, hd) : 0.f;
         }
         __syncthreads();
         for (int e = threadIdx.x; e < KT * kP; e += kThreads) {
@@ -156,7 +156,7 @@ state_scan_kernel(int T, int H, int L, int nc, const CsT* __restrict__ cs,
 template <typename IoT, typename CsT, int N>
 __global__ void __launch_bounds__(kThreads)
 chunk_output_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ x,
-                    const float* __restrict__ dt, const IoT* __restrict__ Bm,
+                    const float* __restrict__ dt, const DtMap dtm, const IoT* __restrict__ Bm,
                     const IoT* __restrict__ Cm, const float* __restrict__ D,
                     const CsT* __restrict__ cs, const float* __restrict__ Hin,
                     IoT* __restrict__ y) {
@@ -229,7 +229,7 @@ chunk_output_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ 
         if (threadIdx.x < TR) {
             const int j = j0 + threadIdx.x;
             s_csj[threadIdx.x] = j < Lc ? csc[j] : CsT(0);
-            s_dtj[threadIdx.x] = j < Lc ? dt[((size_t)bi * T + t0 + j) * H + hd] : 0.f;
+            s_dtj[threadIdx.x] = j < Lc ? dt_value(dt[((size_t)bi * T + t0 + j) * H + hd], dtm, hd) : 0.f;
         }
         __syncthreads();
         // G = C_i . B_j over this 64 x 64 tile
@@ -288,7 +288,7 @@ chunk_output_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ 
 }
 
 template <typename IoT, typename CsT, int N>
-int run(int b, int T, int H, int G, int L, const void* x, const float* dt, const float* A,
+int run(int b, int T, int H, int G, int L, const void* x, const float* dt, const DtMap dtm, const float* A,
         const void* Bm, const void* Cm, const float* D, const float* h0, void* y, float* hf,
         char* ws, cudaStream_t s) {
     const int nc = (T + L - 1) / L;
@@ -300,11 +300,11 @@ int run(int b, int T, int H, int G, int L, const void* x, const float* dt, const
     dim3 gchunk(nc, H, b);
     {
         LaunchScope ls("simt_decay_cumsum", s);
-        decay_cumsum_kernel<CsT><<<gchunk, kThreads, 0, s>>>(T, H, L, nc, dt, A, cs);
+        decay_cumsum_kernel<CsT><<<gchunk, kThreads, 0, s>>>(T, H, L, nc, dt, dtm, A, cs);
     }
     {
         LaunchScope ls("simt_chunk_state", s);
-        chunk_state_kernel<IoT, CsT, N><<<gchunk, kThreads, 0, s>>>(T, H, G, L, nc, xi, dt, Bi, cs, S);
+        chunk_state_kernel<IoT, CsT, N><<<gchunk, kThreads, 0, s>>>(T, H, G, L, nc, xi, dt, dtm, Bi, cs, S);
     }
     {
         LaunchScope ls("simt_state_scan", s);
@@ -315,7 +315,7 @@ int run(int b, int T, int H, int G, int L, const void* x, const float* dt, const
     SSD_CUDA_TRY(cudaFuncSetAttribute(k4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     {
         LaunchScope ls("simt_chunk_output", s);
-        k4<<<dim3(nc * ((L + 63) / 64), H, b), kThreads, smem, s>>>(T, H, G, L, nc, xi, dt, Bi, Ci, D, cs, S,
+        k4<<<dim3(nc * ((L + 63) / 64), H, b), kThreads, smem, s>>>(T, H, G, L, nc, xi, dt, dtm, Bi, Ci, D, cs, S,
                                                                      static_cast<IoT*>(y));
     }
     SSD_CUDA_TRY(cudaGetLastError());
@@ -332,16 +332,16 @@ size_t prefill_simt_workspace_bytes(int b, int T, int H, int N, int L, int io) {
 }
 
 int launch_prefill_simt(int b, int T, int H, int N, int G, int L, int io, const void* x,
-                        const float* dt, const float* A, const void* Bm, const void* Cm,
+                        const float* dt, const DtMap& dtm, const float* A, const void* Bm, const void* Cm,
                         const float* D, const float* h0, void* y, float* hf, void* ws,
                         cudaStream_t s) {
     char* w = static_cast<char*>(ws);
     if (io == SSD_F32) {
-        return N == 128 ? run<float, double, 128>(b, T, H, G, L, x, dt, A, Bm, Cm, D, h0, y, hf, w, s)
-                        : run<float, double, 64>(b, T, H, G, L, x, dt, A, Bm, Cm, D, h0, y, hf, w, s);
+        return N == 128 ? run<float, double, 128>(b, T, H, G, L, x, dt, dtm, A, Bm, Cm, D, h0, y, hf, w, s)
+                        : run<float, double, 64>(b, T, H, G, L, x, dt, dtm, A, Bm, Cm, D, h0, y, hf, w, s);
     }
-    return N == 128 ? run<__nv_bfloat16, float, 128>(b, T, H, G, L, x, dt, A, Bm, Cm, D, h0, y, hf, w, s)
-                    : run<__nv_bfloat16, float, 64>(b, T, H, G, L, x, dt, A, Bm, Cm, D, h0, y, hf, w, s);
+    return N == 128 ? run<__nv_bfloat16, float, 128>(b, T, H, G, L, x, dt, dtm, A, Bm, Cm, D, h0, y, hf, w, s)
+                    : run<__nv_bfloat16, float, 64>(b, T, H, G, L, x, dt, dtm, A, Bm, Cm, D, h0, y, hf, w, s);
 }
 
 }  // namespace ssd

@@ -113,6 +113,7 @@ struct TcParams {
     CUtensorMap tm_C;
     CUtensorMap tm_y;
     const float* dt;
+    DtMap dtm;                   // dt as given, or the softplus pre-processing of raw dt
     const float* A;
     const float* D;
     const float* h0;
@@ -660,7 +661,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         bool stopped = false;
         auto load_dt = [&](int u) {
             const int tok = tb + u * kBlk + r;
-            return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;
+            return (u < nblk && tok < T) ? dt_value(__ldg(prm.dt + ((size_t)bi * T + tok) * H + hd), prm.dtm, hd) : 0.f;
         };
         // dt is fetched two blocks ahead: under full HBM load its latency is microseconds
         float dt_a = load_dt(0), dt_b = load_dt(1);
@@ -885,7 +886,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
         for (int k = 0; k < 32; ++k) Hs[k] = 0.f;
         auto load_dt = [&](int u) {
             const int tok = tb + u * kBlk + r;
-            return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;
+            return (u < nblk && tok < T) ? dt_value(__ldg(prm.dt + ((size_t)bi * T + tok) * H + hd), prm.dtm, hd) : 0.f;
         };
         bool live = __all_sync(0xffffffffu, !*s_abort);
         bool stopped = false;
@@ -1106,7 +1107,8 @@ std::atomic<unsigned long long> g_starve_ns{0};
 void prefill_tc_starve_next(unsigned long long wait_ns) { g_starve_ns.store(wait_ns); }
 void prefill_tc_force_segments(int nseg) { g_force_nseg.store(nseg); }
 
-int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt, const float* A, const void* Bm,
+int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt, const DtMap& dtm, const float* A,
+                      const void* Bm,
                       const void* Cm, const float* D, const float* h0, void* y, float* hf, void* ws,
                       cudaStream_t s) {
     TcParams prm;
@@ -1117,6 +1119,7 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     if ((st = make_map(&prm.tm_C, Cm, kN, G, T, b)) != SSD_OK) return st;
     if ((st = make_map(&prm.tm_y, y, kP, H, T, b)) != SSD_OK) return st;
     prm.dt = dt;
+    prm.dtm = dtm;
     prm.A = A;
     prm.D = D;
     prm.h0 = h0;

@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill_workspace_size.restype = _sz
         L.ssd_prefill.argtypes = [_i] * 8 + [_vp] * 10 + [_sz, _vp]
         L.ssd_prefill.restype = _i
+        L.ssd_prefill_dt_raw.argtypes = [_i] * 8 + [_vp] * 3 + [ctypes.c_float] * 2 + [_vp] * 8 + [_sz, _vp]
+        L.ssd_prefill_dt_raw.restype = _i
         L.ssd_prefill_check.argtypes = [_vp, _vp]
         L.ssd_prefill_check.restype = _i
         L.ssd_debug_starve_next_prefill.argtypes = [ctypes.c_ulonglong]
@@ -150,9 +152,12 @@ def prefill_workspace_size(b, T, H, P, N, G, chunk, io_dtype) -> int:
 
 
 def prefill(x, dt, A, B, C, D, chunk=256, h0=None, y=None, h_final=None, workspace=None,
-            want_final=True, stream=None, check=False):
+            want_final=True, stream=None, check=False, dt_raw=False, dt_bias=None, dt_min=0.0,
+            dt_max=float("inf")):
     """Chunked SSD prefill.  Shapes: x [b,T,H,P], dt [b,T,H] f32, A [H] f32,
     B/C [b,T,G,N], D [H] f32, h0 [b,H,P,N] f32 or None.  Returns (y, h_final).
+    dt_raw=True passes dt as the raw step (ssd_prefill_dt_raw): the kernels form
+    clamp(softplus(dt + dt_bias[h]), dt_min, dt_max) themselves; dt_bias [H] f32 or None.
     check=True synchronises and raises if a device-side wait recorded an error."""
     _need(x, "x")
     io = _io(x)
@@ -172,14 +177,25 @@ def prefill(x, dt, A, B, C, D, chunk=256, h0=None, y=None, h_final=None, workspa
         h_final = torch.empty((b, H, P, N), dtype=torch.float32, device=x.device)
     if h_final is not None:
         _need(h_final, "h_final", torch.float32, (b, H, P, N))
+    if dt_bias is not None:
+        _need(dt_bias, "dt_bias", torch.float32, (H,))
     need = prefill_workspace_size(b, T, H, P, N, G, chunk, io)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().ssd_prefill(b, T, H, P, N, G, int(chunk), io, _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
-                           _ptr(C), _ptr(D), _ptr(h0), _ptr(y), _ptr(h_final), _ptr(workspace),
-                           ws_bytes, _stream(stream))
-    _check(st, "ssd_prefill")
+    if dt_raw:
+        st = lib().ssd_prefill_dt_raw(b, T, H, P, N, G, int(chunk), io, _ptr(x), _ptr(dt), _ptr(dt_bias),
+                                      float(dt_min), float(dt_max), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                      _ptr(h0), _ptr(y), _ptr(h_final), _ptr(workspace), ws_bytes,
+                                      _stream(stream))
+        _check(st, "ssd_prefill_dt_raw")
+    else:
+        if dt_bias is not None:
+            raise ValueError("dt_bias applies to the raw step only (pass dt_raw=True)")
+        st = lib().ssd_prefill(b, T, H, P, N, G, int(chunk), io, _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                               _ptr(C), _ptr(D), _ptr(h0), _ptr(y), _ptr(h_final), _ptr(workspace),
+                               ws_bytes, _stream(stream))
+        _check(st, "ssd_prefill")
     if check and workspace is not None:
         prefill_check(workspace, stream)
     return y, h_final

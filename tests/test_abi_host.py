@@ -186,3 +186,22 @@ def test_starve_hook_rejects_out_of_range_limits():
     L = ssd.lib()
     assert L.ssd_debug_starve_next_prefill(999_999) == 1
     assert L.ssd_debug_starve_next_prefill(10_000_000_001) == 1
+
+
+def test_prefill_dt_raw_rejects_bad_clamp_and_bias():
+    """ssd_prefill_dt_raw validates its clamp range and dt_bias before anything else runs."""
+    L = ssd.lib()
+    x, dt, A, B, C, D, y, ws = _fake(8)
+    bias = ctypes.c_void_p(0x20000000)
+
+    def call(lo, hi, bias_ptr=bias, H=4):
+        return L.ssd_prefill_dt_raw(1, 512, H, 64, 64, 1, 256, 1, x, dt, bias_ptr, lo, hi, A, B, C, D, None, y,
+                                    None, ws, 1 << 30, None)
+    inf, nan = float("inf"), float("nan")
+    for lo, hi in [(-1e-3, 1.0), (0.5, 0.5), (0.5, 0.1), (nan, 1.0), (0.0, nan), (inf, inf)]:
+        assert call(lo, hi) == INVALID, (lo, hi)
+        assert ssd.last_error() != ""
+    assert call(0.0, inf, ctypes.c_void_p(0x20000004)) == INVALID      # misaligned dt_bias
+    # a bad shape is reported as for ssd_prefill
+    assert L.ssd_prefill_dt_raw(1, 512, 6, 64, 64, 4, 256, 1, x, dt, None, 0.0, inf, A, B, C, D, None, y, None, ws,
+                                1 << 30, None) == INVALID

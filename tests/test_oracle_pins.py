@@ -284,3 +284,27 @@ def test_decode_layers_and_rows_independent():
     np.testing.assert_array_equal(y[2:3, 1:2], y1)
     np.testing.assert_array_equal(h[2:3, 1:2], h1)
     np.testing.assert_array_equal(cs[2:3, 1:2], cs1)
+
+
+# ------------------------------------------------------------------ dt pre-processing
+def test_dt_from_raw_closed_forms():
+    """softplus(0) = ln 2; softplus(ln(e^k - 1)) = k; softplus(z) - softplus(-z) = z (the
+    odd part of softplus is z/2); softplus(z) -> z for large z and -> e^z for very negative z."""
+    ks = np.array([0.25, 1.0, 3.0, 10.0])
+    got = oracle.dt_from_raw(np.log(np.expm1(ks))[None, :])
+    np.testing.assert_allclose(got[0], ks, rtol=1e-14)
+    assert abs(oracle.dt_from_raw(np.zeros((1, 1)))[0, 0] - np.log(2.0)) < 1e-15
+    z = np.linspace(-30, 30, 121)[None, :]
+    np.testing.assert_allclose(oracle.dt_from_raw(z) - oracle.dt_from_raw(-z), z, atol=1e-12)
+    np.testing.assert_allclose(oracle.dt_from_raw(np.array([[40.0, 300.0]])), [[40.0, 300.0]], rtol=1e-15)
+    np.testing.assert_allclose(oracle.dt_from_raw(np.array([[-40.0, -600.0]])), np.exp([[-40.0, -600.0]]), rtol=1e-12)
+
+
+def test_dt_from_raw_bias_per_head_and_clamp():
+    """The bias is added per head (last axis) before the softplus; the clamp bounds the result."""
+    raw = np.zeros((2, 3, 4))
+    bias = np.log(np.expm1(np.array([0.001, 0.01, 0.1, 1.0])))
+    got = oracle.dt_from_raw(raw, bias)
+    np.testing.assert_allclose(got, np.broadcast_to([0.001, 0.01, 0.1, 1.0], raw.shape), rtol=1e-12)
+    clamped = oracle.dt_from_raw(raw, bias, dt_min=0.005, dt_max=0.5)
+    np.testing.assert_allclose(clamped[0, 0], [0.005, 0.01, 0.1, 0.5], rtol=1e-12)
