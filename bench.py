@@ -497,8 +497,10 @@ def main():
     clk = clocks.stop()
 
     cpu = None
+    ablation = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(case, flops / (PB * PT * PH))
+        ablation = decay_precision_ablation(ssd, torch, dev)
 
     if rank == 0:
         line = {"metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -513,10 +515,43 @@ def main():
                 "hbm_gbs_alg": pbytes * world / (ms * 1e-3) / 1e9,
                 "tensor_frac": tflops / world / pk["bf16_tflops"],
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
-                "clocks": clk, "decode": decode, "prefill_configs": other, "prefill_dt_raw": dt_raw_entry}
+                "clocks": clk, "decode": decode, "prefill_configs": other, "prefill_dt_raw": dt_raw_entry,
+                "decay_precision_ablation": ablation}
         print(json.dumps(line), flush=True)
     ranks.close()
     return 0
+
+
+def decay_precision_ablation(ssd, torch, dev):
+    """The analogue of the paper's decay-precision table without a model: the 130M-layer
+    prefill (b=1, T=4096, H=24, one pass) with the decay in fp32 (the product), with every
+    exponentiated decay factor rounded to bf16, and with the log-space prefix sums rounded
+    to bf16 before exponentiation; max |error| of y and h_final against the fp64 oracle,
+    also divided by max |reference|.  Not timed."""
+    import oracle
+    from ssd_inputs import make_config
+    c = make_config("mamba2_130m_layer")
+    def bf(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    x, Bm, Cm = bf(c.x_bits), bf(c.B_bits), bf(c.C_bits)
+    dt, A, D = (torch.from_numpy(v).to(dev) for v in (c.dt, c.A, c.D))
+    y_ref, h_ref = oracle.ssd_recurrence(c.x, c.dt, c.A, c.B, c.C, c.D, None)
+    out = {}
+    ssd.debug_force_prefill_segments(1)
+    try:
+        for mode, name in ((0, "fp32_log_space_decay"), (1, "bf16_exp_outputs"), (2, "bf16_log_space_prefix_sums")):
+            ssd.debug_decay_precision(mode)
+            y, hf = ssd.prefill(x, dt, A, Bm, Cm, D, chunk=256)
+            torch.cuda.synchronize()
+            yd = np.abs(y.float().cpu().numpy() - y_ref)
+            hd = np.abs(hf.cpu().numpy() - h_ref)
+            out[name] = {"y_max_abs": float(yd.max()), "y_rel": float(yd.max() / np.abs(y_ref).max()),
+                         "h_max_abs": float(hd.max()), "h_rel": float(hd.max() / np.abs(h_ref).max())}
+    finally:
+        ssd.debug_decay_precision(0)
+        ssd.debug_force_prefill_segments(0)
+    out["workload"] = "mamba2_130m_layer prefill, one pass, bf16 io"
+    return out
 
 
 def bench_prefill_configs(ssd, torch, dev, stream, args, clocks, barrier, max_over_ranks, world, pk, box):

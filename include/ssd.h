@@ -149,6 +149,16 @@ SSD_API int ssd_debug_starve_next_prefill(unsigned long long wait_limit_ns);
  * Errors: SSD_ERR_INVALID_ARG if nseg < 0. */
 SSD_API int ssd_debug_force_prefill_segments(int nseg);
 
+/* Decay-precision ablation for the tensor-core prefill ([CF-SSD] "Precision management":
+ * decay parameters held in log space in fp32 and exponentiated at compute time; bf16 for
+ * the decay exponentiation alone shifts the output).  mode 0 (the default) keeps every
+ * decay quantity in fp32; mode 1 rounds every exponentiated decay factor to bf16; mode 2
+ * rounds the log-space prefix sums of dt*A to bf16 before they are exponentiated.  Applies
+ * to every following tensor-core ssd_prefill in this process until reset with 0.  For
+ * measuring the effect only: modes 1 and 2 are less accurate by design.
+ * Errors: SSD_ERR_INVALID_ARG if mode is not 0, 1 or 2. */
+SSD_API int ssd_debug_decay_precision(int mode);
+
 /* Segments per sequence that ssd_prefill would use for this shape: 1 when the whole
  * sequence runs in one pass (every shape outside the tensor-core path, and tensor-core
  * shapes with enough sequence-heads for the SMs of the current device), else the count of

@@ -11,6 +11,7 @@ from .ssd import (  # noqa: F401
     SSD_F32,
     DecodePlan,
     SSDError,
+    debug_decay_precision,
     debug_force_prefill_segments,
     debug_starve_next_prefill,
     decode_loop,

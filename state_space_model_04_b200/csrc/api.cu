@@ -29,6 +29,7 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
 int prefill_tc_status(void* ws, cudaStream_t s);
 void prefill_tc_starve_next(unsigned long long wait_ns);
 void prefill_tc_force_segments(int nseg);
+void prefill_tc_decay_mode(int mode);
 int prefill_tc_segments(int b, int T, int H);
 size_t decode_workspace_bytes(int layers, int b, int G);
 int launch_decode_step(int layers, int b, int H, int N, int G, int act, int io, float* h,
@@ -220,6 +221,13 @@ int ssd_prefill_segments(int b, int T, int H, int P, int N, int G, int chunk, in
     if (check_prefill_shape(b, T, H, P, N, G, chunk, io_dtype) != SSD_OK) return 0;
     if (b == 0 || T == 0 || !prefill_tc_supported(P, N, io_dtype)) return 1;
     return prefill_tc_segments(b, T, H);
+}
+
+int ssd_debug_decay_precision(int mode) {
+    g_detail[0] = 0;
+    if (mode < 0 || mode > 2) return set_error(SSD_ERR_INVALID_ARG, "decay precision mode %d is not 0, 1 or 2", mode);
+    prefill_tc_decay_mode(mode);
+    return SSD_OK;
 }
 
 int ssd_debug_force_prefill_segments(int nseg) {

@@ -231,6 +231,13 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Decay-precision ablation, a compile-time kernel parameter (kDecay): 0 keeps every decay
+// quantity in fp32 (the product); 1 rounds every exponentiated decay factor to bf16; 2
+// rounds the log-space prefix sums of dt*A to bf16 before they are exponentiated.
+__device__ __forceinline__ float bf16r(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
+template <int kDecay> __device__ __forceinline__ float dlog(float v) { return kDecay == 2 ? bf16r(v) : v; }
+template <int kDecay> __device__ __forceinline__ float dexp(float v) { return kDecay == 1 ? bf16r(v) : v; }
+
 // UMMA shared-memory matrix descriptor: 128-byte swizzle, sm_100 version field.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
@@ -338,6 +345,7 @@ __device__ __forceinline__ float block_cumsum(float a, int q, int lane, bool pub
 }
 
 // ------------------------------------------------------------------ kernel
+template <int kDecay>
 __global__ void __launch_bounds__(kThreads, 1)
 ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -559,7 +567,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 const float* ms = s_m + s * kBlk;
                 const float cs = s_cs[s * kBlk + r];
                 const float csl = cs * kLog2e;
-                ei_cur = __expf(cs);
+                ei_cur = dexp<kDecay>(__expf(cs));
                 float cend[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) cend[c] = s_cend[s * 4 + c];
@@ -580,7 +588,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                     }
                     if (c < q) {  // below the diagonal sub-block: factorised decay
                         const float ce = (c == 0) ? cend[0] : (c == 1) ? cend[1] : cend[2];
-                        const float uu = __expf(cs - ce);
+                        const float uu = dexp<kDecay>(__expf(cs - ce));
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
                             const float4 v4 = *reinterpret_cast<const float4*>(vs + c * 32 + 4 * k);
@@ -596,8 +604,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                         for (int k = 0; k < 16; ++k) {
                             const int j0 = 2 * k, j1 = 2 * k + 1;  // column within the sub-block
                             const float2 m2 = *reinterpret_cast<const float2*>(ms + c * 32 + j0);
-                            float v0 = (j0 <= lane) ? __uint_as_float(raw[j0]) * ex2(csl + m2.x) : 0.f;
-                            float v1 = (j1 <= lane) ? __uint_as_float(raw[j1]) * ex2(csl + m2.y) : 0.f;
+                            float v0 = (j0 <= lane) ? __uint_as_float(raw[j0]) * dexp<kDecay>(ex2(csl + m2.x)) : 0.f;
+                            float v1 = (j1 <= lane) ? __uint_as_float(raw[j1]) * dexp<kDecay>(ex2(csl + m2.y)) : 0.f;
                             if (j0 == lane) v0 += Dh;
                             if (j1 == lane) v1 += Dh;
                             pk[cc][k] = pack_bf16(v0, v1);
@@ -674,7 +682,13 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             dt_b = load_dt(k + 3);
             if (!live || *s_abort) s_ystop[s] = 1;
             float cend[4], cs_last;
-            const float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_ytot + s * 4, 3, cs_last, cend);
+            float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_ytot + s * 4, 3, cs_last, cend);
+            if (kDecay == 2) {
+                cs = dlog<kDecay>(cs);
+                cs_last = dlog<kDecay>(cs_last);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) cend[c] = dlog<kDecay>(cend[c]);
+            }
             if (s_ystop[s]) { stopped = true; break; }
             // ---- w o X of block k+1 (needs S^T(k) accumulated: the MMA has read Xs(k))
             if (live && k >= 0) live = warp_wait(bar(BAR_ACCS), k & 1, s_abort, prm.status, 13);
@@ -684,7 +698,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 if (half == 0) {
                     s_cs[s * kBlk + r] = cs;
                     s_m[s * kBlk + r] = __log2f(dtv) - cs * kLog2e;   // -inf where dt = 0
-                    s_v[s * kBlk + r] = __expf(cend[q] - cs) * dtv;    // cend[q]: end of j's 32-token group
+                    s_v[s * kBlk + r] = dexp<kDecay>(__expf(cend[q] - cs)) * dtv;  // cend[q]: end of j's group
                     if (r < 4) s_cend[s * 4 + r] = cend[r];
                 }
                 mbar_arrive(bar(BAR_PREP0 + s));
@@ -696,7 +710,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                     uint32_t raw[32];
                     SSD_TMEM_LD32(tmem + lane_addr + kColS + p0, raw);
                     tmem_wait_ld();
-                    const float gam = __expf(cs_last_prev);
+                    const float gam = dexp<kDecay>(__expf(cs_last_prev));
 #pragma unroll
                     for (int j = 0; j < 32; ++j) Hs[j] = fmaf(gam, Hs[j], __uint_as_float(raw[j]));
                 }
@@ -716,7 +730,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 live = warp_wait(bar(BAR_FULLX + (k + 1) % 3), ((k + 1) / 3) & 1, s_abort, prm.status, 14);
                 if (live) {
                     // w_j x_j as one packed bf16x2 multiply per element pair
-                    const __nv_bfloat162 w2 = __float2bfloat162_rn(__expf(cs_last - cs) * dtv);
+                    const __nv_bfloat162 w2 = __float2bfloat162_rn(dexp<kDecay>(__expf(cs_last - cs)) * dtv);
                     const uint8_t* src = smem + kXRing + ((k + 1) % 3) * kRegion;
                     uint8_t* dst = smem + kXs;
 #pragma unroll
@@ -791,6 +805,7 @@ constexpr uint32_t kSSmemBytes = kSSmall + 1024;
 constexpr uint32_t kSTmemCols = 128;                 // two 64-column S buffers
 enum { SB_FULL = 0, SB_EMPTY = 2, SB_XS = 4, SB_ACC = 6, SB_SFREE = 8, SB_DONE = 10, SB_COUNT };
 
+template <int kDecay>
 __global__ void __launch_bounds__(kSThreads, 2)
 ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -900,7 +915,9 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
             dt_b = load_dt(u + 2);
             if (!live || *s_abort) s_ystop[s] = 1;
             float cend[4], cs_last;
-            const float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_tot + s * 4, 4, cs_last, cend);
+            float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_tot + s * 4, 4, cs_last, cend);
+            cs = dlog<kDecay>(cs);
+            cs_last = dlog<kDecay>(cs_last);
             if (s_ystop[s]) {
                 stopped = true;
                 break;
@@ -909,7 +926,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
                 live = warp_wait(bar(SB_FULL + s), (u >> 1) & 1, s_abort, prm.status, 44);
                 if (live) {
                     // w_j x_j in place, one packed bf16x2 multiply per element pair
-                    const __nv_bfloat162 w2 = __float2bfloat162_rn(__expf(cs_last - cs) * dtv);
+                    const __nv_bfloat162 w2 = __float2bfloat162_rn(dexp<kDecay>(__expf(cs_last - cs)) * dtv);
                     uint8_t* xs = smem + s * kSSlot + kSX;
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
@@ -934,7 +951,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
                     tmem_wait_ld();
                     tc_fence_before();
                     mbar_arrive(bar(SB_SFREE + sp));
-                    const float gam = __expf(cs_last_prev);
+                    const float gam = dexp<kDecay>(__expf(cs_last_prev));
 #pragma unroll
                     for (int j = 0; j < 32; ++j) Hs[j] = fmaf(gam, Hs[j], __uint_as_float(raw[j]));
                 }
@@ -1055,6 +1072,7 @@ constexpr double kCtaStartBlocks = 2.0;
 constexpr double kScanPerSegment = 0.4;
 constexpr double kSplitFixedBlocks = 5.0;
 std::atomic<int> g_force_nseg{0};
+std::atomic<int> g_decay_mode{0};
 void plan_segments(int b, int T, int H, int* nseg, int* tseg) {
     const int nb = (T + kBlk - 1) / kBlk;
     if (const int f = g_force_nseg.load()) {
@@ -1106,6 +1124,7 @@ std::atomic<unsigned long long> g_starve_ns{0};
 }
 void prefill_tc_starve_next(unsigned long long wait_ns) { g_starve_ns.store(wait_ns); }
 void prefill_tc_force_segments(int nseg) { g_force_nseg.store(nseg); }
+void prefill_tc_decay_mode(int mode) { g_decay_mode.store(mode); }
 
 int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt, const DtMap& dtm, const float* A,
                       const void* Bm,
@@ -1120,6 +1139,11 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     if ((st = make_map(&prm.tm_y, y, kP, H, T, b)) != SSD_OK) return st;
     prm.dt = dt;
     prm.dtm = dtm;
+    const int decay = g_decay_mode.load();
+    auto fused = decay == 1 ? ssd_prefill_fused_kernel<1> : decay == 2 ? ssd_prefill_fused_kernel<2>
+                                                                        : ssd_prefill_fused_kernel<0>;
+    auto state = decay == 1 ? ssd_segment_state_kernel<1> : decay == 2 ? ssd_segment_state_kernel<2>
+                                                                        : ssd_segment_state_kernel<0>;
     prm.A = A;
     prm.D = D;
     prm.h0 = h0;
@@ -1140,11 +1164,10 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     SSD_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), s));
     if (prm.nseg > 1) {
         // local end states of all segments but the last, then their scan
-        SSD_CUDA_TRY(cudaFuncSetAttribute(ssd_segment_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)kSSmemBytes));
+        SSD_CUDA_TRY(cudaFuncSetAttribute(state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSSmemBytes));
         {
             LaunchScope ls("ssd_segment_state", s);
-            ssd_segment_state_kernel<<<dim3(H, b, prm.nseg - 1), kSThreads, kSSmemBytes, s>>>(prm);
+            state<<<dim3(H, b, prm.nseg - 1), kSThreads, kSSmemBytes, s>>>(prm);
         }
         SSD_CUDA_TRY(cudaGetLastError());
         {
@@ -1154,11 +1177,10 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
         }
         SSD_CUDA_TRY(cudaGetLastError());
     }
-    SSD_CUDA_TRY(cudaFuncSetAttribute(ssd_prefill_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)kSmemBytes));
+    SSD_CUDA_TRY(cudaFuncSetAttribute(fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes));
     {
         LaunchScope ls("ssd_prefill_fused", s);
-        ssd_prefill_fused_kernel<<<dim3(H, b, prm.nseg), kThreads, kSmemBytes, s>>>(prm);
+        fused<<<dim3(H, b, prm.nseg), kThreads, kSmemBytes, s>>>(prm);
     }
     SSD_CUDA_TRY(cudaGetLastError());
     return SSD_OK;

@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_debug_starve_next_prefill.restype = _i
         L.ssd_prefill_segments.argtypes = [_i] * 8
         L.ssd_prefill_segments.restype = _i
+        L.ssd_debug_decay_precision.argtypes = [_i]
+        L.ssd_debug_decay_precision.restype = _i
         L.ssd_debug_force_prefill_segments.argtypes = [_i]
         L.ssd_debug_force_prefill_segments.restype = _i
         L.ssd_decode_workspace_size.argtypes = [_i] * 3
@@ -215,6 +217,12 @@ def debug_starve_next_prefill(wait_limit_s=0.1):
 def prefill_segments(b, T, H, P, N, G, chunk, io_dtype) -> int:
     """Segments per sequence ssd_prefill uses for this shape (1 = one pass; 0 = invalid)."""
     return int(lib().ssd_prefill_segments(b, T, H, P, N, G, chunk, io_dtype))
+
+
+def debug_decay_precision(mode=0):
+    """Decay-precision ablation of the tensor-core prefill: 0 fp32 (default), 1 exponentiated
+    decay factors rounded to bf16, 2 log-space prefix sums rounded to bf16 before exp."""
+    _check(lib().ssd_debug_decay_precision(int(mode)), "ssd_debug_decay_precision")
 
 
 def debug_force_prefill_segments(nseg=0):

@@ -181,6 +181,12 @@ def test_segment_hook_and_workspace():
         ssd.debug_force_prefill_segments(0)
 
 
+def test_decay_precision_hook_rejects_unknown_modes():
+    L = ssd.lib()
+    assert L.ssd_debug_decay_precision(3) == INVALID and L.ssd_debug_decay_precision(-1) == INVALID
+    assert L.ssd_debug_decay_precision(0) == OK
+
+
 def test_starve_hook_rejects_out_of_range_limits():
     import state_space_model_04_b200 as ssd
     L = ssd.lib()

@@ -320,3 +320,29 @@ def test_dt_raw_equals_preprocessed_dt():
     torch.cuda.synchronize()
     check(_np(y_raw), _np(y_pre), "bf16", "y raw vs pre-processed")
     check(_np(h_raw), _np(h_pre), "bf16", "h_final raw vs pre-processed")
+
+
+# ------------------------------------------------------------------ decay precision ablation
+def test_decay_precision_ablation():
+    """Holding the decay in log space in fp32 matters ("Precision management" of the paper):
+    rounding the log-space prefix sums to bf16 before exponentiating (mode 2) costs far more
+    accuracy than rounding each exponentiated factor (mode 1), and the product's fp32 decay
+    (mode 0) is the most accurate of the three and within the bf16 bound."""
+    case = make_prefill(1, 2048, 8, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=41)
+    errs = {}
+    ssd.debug_force_prefill_segments(1)
+    try:
+        for mode in (0, 1, 2):
+            ssd.debug_decay_precision(mode)
+            y, hf, _ = run_prefill(ssd, case)
+            torch.cuda.synchronize()
+            errs[mode] = (_np(y), _np(hf))
+    finally:
+        ssd.debug_decay_precision(0)
+        ssd.debug_force_prefill_segments(0)
+    y_ref, hf_ref = oracle_subset(case, [0], range(case.H))
+    e = {m: (rel_max(v[0], y_ref), rel_max(v[1], hf_ref)) for m, v in errs.items()}
+    print("decay precision ablation (y, h_final) max-normalised error:", e)
+    assert e[0][0] <= 2e-2 and e[0][1] <= 2e-2
+    assert e[0][0] <= e[1][0] * 1.5 and e[1][0] < e[2][0]
+    assert e[2][0] > 2 * e[0][0]
