@@ -123,6 +123,49 @@ SSD_API int ssd_prefill_dt_raw(int b, int T, int H, int P, int N, int G, int chu
                        const float* h0, void* y, float* h_final, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------------------
+ * Context-parallel prefill: one sequence's tokens split over ranks  ([CF-SSD] "Chunked
+ * recurrence": the state entering a stretch of tokens is the decayed sum of the states the
+ * earlier stretches leave behind, and y is linear in that state)
+ *
+ * Rank r holds the consecutive tokens [T_0 + ... + T_{r-1}, ... + T_r) of every sequence.
+ *   1. ssd_prefill_local_state: the state its tokens leave when started from zero, and
+ *      their total log decay sum(dt * A), per (sequence, head);
+ *   2. the caller all-gathers both across ranks, rank-major (one NCCL all-gather each);
+ *   3. ssd_prefill_context_scan: the state entering this rank's tokens;
+ *   4. ssd_prefill with h0 = that state: this rank's y and the state after its tokens (the
+ *      whole sequence's final state on the last rank).
+ * The result equals one ssd_prefill over the whole sequence up to rounding.
+ * ---------------------------------------------------------------------------------- */
+
+/* Workspace bytes for ssd_prefill_local_state (0 for shapes it does not take or b == 0 or
+ * T == 0). */
+SSD_API size_t ssd_prefill_local_state_workspace_size(int b, int T, int H, int P, int N, int G,
+                                                      int io_dtype);
+
+/* Step 1.  x [b][T][H][P] bf16, dt [b][T][H] fp32 (positive), A [H] fp32, B [b][T][G][N] bf16 as
+ * for ssd_prefill; outputs h_local [b][H][P][N] fp32 (the recurrence over these T tokens
+ * from h = 0) and log_decay [b][H] fp32 (sum over the tokens of dt * A).  Runs the
+ * tensor-core state pass (the tokens cut into pieces to fill the SMs) and a fold of the
+ * pieces.  T == 0 writes zeros.  Tensor-core shapes only: bf16, P = 64, N = 128.
+ * Errors: SSD_ERR_INVALID_ARG (bad shape or pointer, outputs overlapping inputs or each
+ * other), SSD_ERR_UNSUPPORTED (other dtypes or P, N), SSD_ERR_WORKSPACE, SSD_ERR_CUDA. */
+SSD_API int ssd_prefill_local_state(int b, int T, int H, int P, int N, int G, int io_dtype,
+                                    const void* x, const float* dt, const float* A, const void* B,
+                                    float* h_local, float* log_decay, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* Step 3.  h_local_all [world][b][H][P][N] and log_decay_all [world][b][H] (fp32, as
+ * all-gathered, rank-major); h0 [b][H][P][N] the state before the first rank's tokens (NULL:
+ * zeros).  Writes h_in [b][H][P][N] = the state entering rank `rank`'s tokens:
+ *   run = h0; for q < rank: run = exp(log_decay_all[q]) * run + h_local_all[q].
+ * Only ranks q < rank are read (may be NULL for rank 0).  h_in may alias h0 exactly.
+ * Errors: SSD_ERR_INVALID_ARG (rank outside [0, world), b < 0, H < 1, bad pointers or
+ * overlaps), SSD_ERR_UNSUPPORTED (P != 64 or N != 128), SSD_ERR_CUDA. */
+SSD_API int ssd_prefill_context_scan(int world, int rank, int b, int H, int P, int N,
+                                     const float* h0, const float* h_local_all,
+                                     const float* log_decay_all, float* h_in, void* stream);
+
 /* Synchronises `stream` and returns the device-side status recorded by the most recent
  * ssd_prefill that used `workspace` (SSD_OK, or SSD_ERR_TIMEOUT if a bounded wait inside
  * the tensor-core kernel expired, or SSD_ERR_INTERNAL for a failed device consistency

@@ -25,6 +25,8 @@ from .ssd import (  # noqa: F401
     profile_end,
     prefill,
     prefill_check,
+    prefill_context_scan,
+    prefill_local_state,
     prefill_segments,
     prefill_workspace_size,
     status_string,

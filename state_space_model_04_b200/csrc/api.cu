@@ -31,6 +31,11 @@ void prefill_tc_starve_next(unsigned long long wait_ns);
 void prefill_tc_force_segments(int nseg);
 void prefill_tc_decay_mode(int mode);
 int prefill_tc_segments(int b, int T, int H);
+size_t prefill_tc_local_state_workspace_bytes(int b, int T, int H);
+int launch_prefill_tc_local_state(int b, int T, int H, int G, const void* x, const float* dt, const float* A,
+                                  const void* Bm, float* h_local, float* log_decay, void* ws, cudaStream_t s);
+int launch_context_scan(int rank, int b, int H, const float* h0, const float* h_all, const float* ld_all,
+                        float* h_in, cudaStream_t s);
 size_t decode_workspace_bytes(int layers, int b, int G);
 int launch_decode_step(int layers, int b, int H, int N, int G, int act, int io, float* h,
                        float* conv_state, const void* xbc, const float* dt, const float* A,
@@ -221,6 +226,74 @@ int ssd_prefill_segments(int b, int T, int H, int P, int N, int G, int chunk, in
     if (check_prefill_shape(b, T, H, P, N, G, chunk, io_dtype) != SSD_OK) return 0;
     if (b == 0 || T == 0 || !prefill_tc_supported(P, N, io_dtype)) return 1;
     return prefill_tc_segments(b, T, H);
+}
+
+size_t ssd_prefill_local_state_workspace_size(int b, int T, int H, int P, int N, int G, int io_dtype) {
+    if (check_prefill_shape(b, T, H, P, N, G, 256, io_dtype) != SSD_OK || !prefill_tc_supported(P, N, io_dtype))
+        return 0;
+    if (b == 0 || T == 0) return 0;
+    return prefill_tc_local_state_workspace_bytes(b, T, H);
+}
+
+int ssd_prefill_local_state(int b, int T, int H, int P, int N, int G, int io_dtype, const void* x, const float* dt,
+                            const float* A, const void* B, float* h_local, float* log_decay, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    g_detail[0] = 0;
+    SSD_CHECK(check_prefill_shape(b, T, H, P, N, G, 256, io_dtype));
+    if (!prefill_tc_supported(P, N, io_dtype))
+        return set_error(SSD_ERR_UNSUPPORTED, "local state: tensor-core shapes only (bf16, P = 64, N = 128)");
+    SSD_CHECK(check_ptr(h_local, "h_local", true));
+    SSD_CHECK(check_ptr(log_decay, "log_decay", true));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t state_bytes = (size_t)b * H * P * N * sizeof(float), ld_bytes = (size_t)b * H * sizeof(float);
+    if (overlaps({h_local, state_bytes}, {log_decay, ld_bytes}))
+        return set_error(SSD_ERR_INVALID_ARG, "h_local overlaps log_decay");
+    if (b == 0) return SSD_OK;
+    if (T == 0) {  // no tokens: nothing accumulates and nothing decays
+        SSD_CUDA_TRY(cudaMemsetAsync(h_local, 0, state_bytes, s));
+        SSD_CUDA_TRY(cudaMemsetAsync(log_decay, 0, ld_bytes, s));
+        return SSD_OK;
+    }
+    SSD_CHECK(check_ptr(x, "x", true));
+    SSD_CHECK(check_ptr(dt, "dt", true));
+    SSD_CHECK(check_ptr(A, "A", true));
+    SSD_CHECK(check_ptr(B, "B", true));
+    const Range outs[] = {{h_local, state_bytes}, {log_decay, ld_bytes}};
+    const Range rin[] = {{x, (size_t)b * T * H * P * 2}, {B, (size_t)b * T * G * N * 2}, {dt, (size_t)b * T * H * 4},
+                         {A, (size_t)H * 4}};
+    for (const Range& o : outs)
+        for (const Range& i : rin)
+            if (overlaps(o, i)) return set_error(SSD_ERR_INVALID_ARG, "an output overlaps an input");
+    const size_t need = prefill_tc_local_state_workspace_bytes(b, T, H);
+    if (!workspace || workspace_bytes < need)
+        return set_error(SSD_ERR_WORKSPACE, "workspace %zu bytes at %p, need %zu", workspace_bytes, workspace, need);
+    if (!aligned16(workspace)) return set_error(SSD_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    for (const Range& o : outs)
+        if (overlaps({workspace, need}, o)) return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps an output");
+    return launch_prefill_tc_local_state(b, T, H, G, x, dt, A, B, h_local, log_decay, workspace, s);
+}
+
+int ssd_prefill_context_scan(int world, int rank, int b, int H, int P, int N, const float* h0, const float* h_local_all,
+                             const float* log_decay_all, float* h_in, void* stream) {
+    g_detail[0] = 0;
+    if (world < 1 || rank < 0 || rank >= world)
+        return set_error(SSD_ERR_INVALID_ARG, "rank %d outside [0, world=%d)", rank, world);
+    if (b < 0 || H < 1) return set_error(SSD_ERR_INVALID_ARG, "b=%d H=%d", b, H);
+    if (P != 64 || N != 128) return set_error(SSD_ERR_UNSUPPORTED, "context scan: P = 64, N = 128 only");
+    if (H > kMaxGridYZ || b > kMaxGridYZ) return set_error(SSD_ERR_UNSUPPORTED, "H=%d or b=%d above 65535", H, b);
+    SSD_CHECK(check_ptr(h0, "h0", false));
+    SSD_CHECK(check_ptr(h_in, "h_in", true));
+    if (rank > 0) {
+        SSD_CHECK(check_ptr(h_local_all, "h_local_all", true));
+        SSD_CHECK(check_ptr(log_decay_all, "log_decay_all", true));
+    }
+    const size_t state_bytes = (size_t)b * H * P * N * sizeof(float);
+    if (overlaps({h_in, state_bytes}, {h_local_all, (size_t)world * state_bytes}) ||
+        overlaps({h_in, state_bytes}, {log_decay_all, (size_t)world * b * H * 4}) ||
+        (h0 && h0 != h_in && overlaps({h_in, state_bytes}, {h0, state_bytes})))
+        return set_error(SSD_ERR_INVALID_ARG, "h_in overlaps an input (only exact aliasing of h0 is allowed)");
+    if (b == 0) return SSD_OK;
+    return launch_context_scan(rank, b, H, h0, h_local_all, log_decay_all, h_in, static_cast<cudaStream_t>(stream));
 }
 
 int ssd_debug_decay_precision(int mode) {

@@ -1013,6 +1013,47 @@ __global__ void __launch_bounds__(kScanThreads) ssd_segment_scan_kernel(const fl
     }
 }
 
+// Folds consecutive stretches of one sequence into one state, per (sequence, head) u:
+// run = h0 (or 0); for q in [0, n): run = exp(logdecay_q) run + h_q; out = run, and
+// out_logdecay = sum of logdecay_q (when given).  Stretch q of unit u = bi * H + hd sits at
+// st + q * st_q + u * st_u (P x N fp32), its log decay at ld + q * ld_q + u * ld_u (strides
+// in elements).  Serves the context-parallel prefill (the stretches: the ranks before this
+// one, rank-major) and the local state of a stretch computed in pieces (unit-major).
+__global__ void __launch_bounds__(kScanThreads) ssd_state_fold_kernel(const float* h0, const float* st, size_t st_q,
+                                                                       size_t st_u, const float* ld, size_t ld_q,
+                                                                       size_t ld_u, int n, int H, float* out,
+                                                                       float* out_logdecay) {
+    const int hd = blockIdx.x, bi = blockIdx.y;
+    const size_t u = (size_t)bi * H + hd;
+    const int e0 = blockIdx.z * (kP * kN / kScanSplit) + threadIdx.x;
+    float run[kScanPer];
+#pragma unroll
+    for (int k = 0; k < kScanPer; ++k) run[k] = h0 ? h0[u * kP * kN + e0 + kScanThreads * k] : 0.f;
+    float ldsum = 0.f;
+    for (int q0 = 0; q0 < n; q0 += kScanBatch) {
+        float v[kScanBatch][kScanPer], gam[kScanBatch];
+#pragma unroll
+        for (int j = 0; j < kScanBatch; ++j) {
+            const bool in = q0 + j < n;
+            const float l = in ? ld[(q0 + j) * ld_q + u * ld_u] : 0.f;
+            ldsum += l;
+            gam[j] = __expf(l);
+            const float* w = st + (q0 + j) * st_q + u * st_u;
+#pragma unroll
+            for (int k = 0; k < kScanPer; ++k) v[j][k] = in ? w[e0 + kScanThreads * k] : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < kScanBatch; ++j) {
+            if (q0 + j >= n) break;
+#pragma unroll
+            for (int k = 0; k < kScanPer; ++k) run[k] = fmaf(gam[j], run[k], v[j][k]);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kScanPer; ++k) out[u * kP * kN + e0 + kScanThreads * k] = run[k];
+    if (out_logdecay && blockIdx.z == 0 && threadIdx.x == 0) out_logdecay[u] = ldsum;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -1182,6 +1223,77 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
         LaunchScope ls("ssd_prefill_fused", s);
         fused<<<dim3(H, b, prm.nseg), kThreads, kSmemBytes, s>>>(prm);
     }
+    SSD_CUDA_TRY(cudaGetLastError());
+    return SSD_OK;
+}
+
+// Local end state of a stretch of tokens started from zero, and its total log decay (the
+// context-parallel prefill's first step).  The stretch is cut into pieces so that the
+// state pass fills the SMs; the pieces' states are then folded in order.
+namespace {
+int local_pieces(int b, int T, int H) {
+    const int nb = (T + kBlk - 1) / kBlk;
+    const int want = (int)std::ceil(4.0 * sm_count() / std::max(1.0, (double)b * H));  // two waves of 2 CTAs/SM
+    return std::max(1, std::min(nb, want));
+}
+}  // namespace
+
+size_t prefill_tc_local_state_workspace_bytes(int b, int T, int H) {
+    const int n = local_pieces(b, T, H);
+    const size_t units = (size_t)b * H * n;
+    return kSegOffset + align256(units * kP * kN * sizeof(float)) + align256(units * sizeof(float));
+}
+
+int launch_prefill_tc_local_state(int b, int T, int H, int G, const void* x, const float* dt, const float* A,
+                                  const void* Bm, float* h_local, float* log_decay, void* ws, cudaStream_t s) {
+    TcParams prm;
+    memset(&prm, 0, sizeof(prm));
+    int st;
+    if ((st = make_map(&prm.tm_x, x, kP, H, T, b)) != SSD_OK) return st;
+    if ((st = make_map(&prm.tm_B, Bm, kN, G, T, b)) != SSD_OK) return st;
+    prm.dt = dt;
+    prm.dtm = DtMap{nullptr, 0.f, 0.f, 0};
+    prm.A = A;
+    prm.status = reinterpret_cast<int*>(ws);
+    prm.T = T;
+    prm.H = H;
+    prm.G = G;
+    const int n = local_pieces(b, T, H);
+    const int nb = (T + kBlk - 1) / kBlk;
+    prm.tseg = ((nb + n - 1) / n) * kBlk;
+    const int pieces = (T + prm.tseg - 1) / prm.tseg;
+    prm.nseg = pieces + 1;  // the state pass writes pieces 0 .. nseg-2, i.e. every piece
+    const size_t units = (size_t)b * H * pieces;
+    prm.seg_state = reinterpret_cast<float*>(static_cast<char*>(ws) + kSegOffset);
+    prm.seg_logdecay = reinterpret_cast<float*>(static_cast<char*>(ws) + kSegOffset +
+                                                align256(units * kP * kN * sizeof(float)));
+    prm.wait_ns = kWaitLimitNs;
+    SSD_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), s));
+    SSD_CUDA_TRY(cudaFuncSetAttribute(ssd_segment_state_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kSSmemBytes));
+    {
+        LaunchScope ls("ssd_segment_state", s);
+        ssd_segment_state_kernel<0><<<dim3(H, b, pieces), kSThreads, kSSmemBytes, s>>>(prm);
+    }
+    SSD_CUDA_TRY(cudaGetLastError());
+    // piece q of unit u: state at (u * pieces + q) * P * N, log decay at u * pieces + q
+    {
+        LaunchScope ls("ssd_state_fold", s);
+        ssd_state_fold_kernel<<<dim3(H, b, kScanSplit), kScanThreads, 0, s>>>(
+            nullptr, prm.seg_state, (size_t)kP * kN, (size_t)pieces * kP * kN, prm.seg_logdecay, 1, (size_t)pieces,
+            pieces, H, h_local, log_decay);
+    }
+    SSD_CUDA_TRY(cudaGetLastError());
+    return SSD_OK;
+}
+
+// Entering state of context shard `rank` from the gathered local states and log decays of
+// all shards, rank-major ([world][b][H][P][N], [world][b][H]).
+int launch_context_scan(int rank, int b, int H, const float* h0, const float* h_all, const float* ld_all,
+                        float* h_in, cudaStream_t s) {
+    LaunchScope ls("ssd_state_fold", s);
+    ssd_state_fold_kernel<<<dim3(H, b, kScanSplit), kScanThreads, 0, s>>>(
+        h0, h_all, (size_t)b * H * kP * kN, (size_t)kP * kN, ld_all, (size_t)b * H, 1, rank, H, h_in, nullptr);
     SSD_CUDA_TRY(cudaGetLastError());
     return SSD_OK;
 }

@@ -59,6 +59,12 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill_check.restype = _i
         L.ssd_debug_starve_next_prefill.argtypes = [ctypes.c_ulonglong]
         L.ssd_debug_starve_next_prefill.restype = _i
+        L.ssd_prefill_local_state_workspace_size.argtypes = [_i] * 7
+        L.ssd_prefill_local_state_workspace_size.restype = _sz
+        L.ssd_prefill_local_state.argtypes = [_i] * 7 + [_vp] * 7 + [_sz, _vp]
+        L.ssd_prefill_local_state.restype = _i
+        L.ssd_prefill_context_scan.argtypes = [_i] * 6 + [_vp] * 5
+        L.ssd_prefill_context_scan.restype = _i
         L.ssd_prefill_segments.argtypes = [_i] * 8
         L.ssd_prefill_segments.restype = _i
         L.ssd_debug_decay_precision.argtypes = [_i]
@@ -212,6 +218,49 @@ def debug_starve_next_prefill(wait_limit_s=0.1):
     """Failure-detection test hook: the next tensor-core prefill issues no loads, so its
     bounded waits expire after `wait_limit_s` and prefill_check raises SSD_ERR_TIMEOUT."""
     _check(lib().ssd_debug_starve_next_prefill(int(wait_limit_s * 1e9)), "ssd_debug_starve_next_prefill")
+
+
+def prefill_local_state(x, dt, A, B, h_local=None, log_decay=None, workspace=None, stream=None):
+    """The state these tokens leave when started from zero, and their total log decay
+    sum(dt * A), per (sequence, head): returns (h_local [b,H,P,N] f32, log_decay [b,H] f32).
+    x [b,T,H,P] bf16, dt [b,T,H] f32, A [H] f32, B [b,T,G,N] bf16 (ssd_prefill_local_state)."""
+    _need(x, "x", torch.bfloat16)
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    _need(dt, "dt", torch.float32, (b, T, H))
+    _need(A, "A", torch.float32, (H,))
+    _need(B, "B", x.dtype, (b, T, G, N))
+    if h_local is None:
+        h_local = torch.empty((b, H, P, N), dtype=torch.float32, device=x.device)
+    if log_decay is None:
+        log_decay = torch.empty((b, H), dtype=torch.float32, device=x.device)
+    _need(h_local, "h_local", torch.float32, (b, H, P, N))
+    _need(log_decay, "log_decay", torch.float32, (b, H))
+    need = int(lib().ssd_prefill_local_state_workspace_size(b, T, H, P, N, G, SSD_BF16))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().ssd_prefill_local_state(b, T, H, P, N, G, SSD_BF16, _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                                       _ptr(h_local), _ptr(log_decay), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "ssd_prefill_local_state")
+    return h_local, log_decay
+
+
+def prefill_context_scan(rank, h_local_all, log_decay_all, h0=None, h_in=None, stream=None):
+    """State entering context shard `rank` from the rank-major gathered local states
+    [world,b,H,P,N] and log decays [world,b,H] (ssd_prefill_context_scan)."""
+    world, b, H, P, N = h_local_all.shape
+    _need(h_local_all, "h_local_all", torch.float32)
+    _need(log_decay_all, "log_decay_all", torch.float32, (world, b, H))
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (b, H, P, N))
+    if h_in is None:
+        h_in = torch.empty((b, H, P, N), dtype=torch.float32, device=h_local_all.device)
+    _need(h_in, "h_in", torch.float32, (b, H, P, N))
+    st = lib().ssd_prefill_context_scan(world, int(rank), b, H, P, N, _ptr(h0), _ptr(h_local_all),
+                                        _ptr(log_decay_all), _ptr(h_in), _stream(stream))
+    _check(st, "ssd_prefill_context_scan")
+    return h_in
 
 
 def prefill_segments(b, T, H, P, N, G, chunk, io_dtype) -> int:

@@ -211,3 +211,23 @@ def test_prefill_dt_raw_rejects_bad_clamp_and_bias():
     # a bad shape is reported as for ssd_prefill
     assert L.ssd_prefill_dt_raw(1, 512, 6, 64, 64, 4, 256, 1, x, dt, None, 0.0, inf, A, B, C, D, None, y, None, ws,
                                 1 << 30, None) == INVALID
+
+
+def test_context_parallel_entry_points_reject():
+    L = ssd.lib()
+    p = _fake(4)
+    # context scan: rank outside [0, world), shapes it does not take
+    assert L.ssd_prefill_context_scan(2, 2, 1, 4, 64, 128, None, p[0], p[1], p[2], None) == INVALID
+    assert L.ssd_prefill_context_scan(2, -1, 1, 4, 64, 128, None, p[0], p[1], p[2], None) == INVALID
+    assert L.ssd_prefill_context_scan(0, 0, 1, 4, 64, 128, None, p[0], p[1], p[2], None) == INVALID
+    assert L.ssd_prefill_context_scan(2, 1, 1, 4, 64, 64, None, p[0], p[1], p[2], None) == UNSUP
+    assert L.ssd_prefill_context_scan(2, 1, 1, 4, 64, 128, None, None, p[1], p[2], None) == INVALID
+    assert L.ssd_prefill_context_scan(2, 1, 1, 4, 64, 128, None, p[0], p[1], None, None) == INVALID
+    # local state: tensor-core shapes only, outputs required, workspace sized
+    x, dt, A, B, hl, ld, ws = _fake(7)
+    assert L.ssd_prefill_local_state(1, 512, 4, 64, 64, 1, 1, x, dt, A, B, hl, ld, ws, 1 << 30, None) == UNSUP
+    assert L.ssd_prefill_local_state(1, 512, 4, 64, 128, 1, 0, x, dt, A, B, hl, ld, ws, 1 << 30, None) == UNSUP
+    assert L.ssd_prefill_local_state(1, 512, 4, 64, 128, 1, 1, x, dt, A, B, None, ld, ws, 1 << 30, None) == INVALID
+    assert L.ssd_prefill_local_state(1, 512, 4, 64, 128, 1, 1, x, dt, A, B, hl, ld, ws, 16, None) == WS
+    assert ssd.lib().ssd_prefill_local_state_workspace_size(1, 512, 4, 64, 128, 1, 1) > 0
+    assert ssd.lib().ssd_prefill_local_state_workspace_size(1, 512, 4, 64, 64, 1, 1) == 0

@@ -346,3 +346,38 @@ def test_decay_precision_ablation():
     assert e[0][0] <= 2e-2 and e[0][1] <= 2e-2
     assert e[0][0] <= e[1][0] * 1.5 and e[1][0] < e[2][0]
     assert e[2][0] > 2 * e[0][0]
+
+
+# ------------------------------------------------------------------ context-parallel prefill
+@pytest.mark.parametrize("bounds", [[0, 700, 1500], [0, 128, 900, 1001, 1500]])
+def test_context_parallel_emulated(bounds):
+    """The context-parallel steps with the ranks emulated in one process (the all-gather
+    replaced by stacking): each shard's local state and log decay (tensor-core state pass
+    and fold), each rank's entering state (fold of the earlier ranks), the prefill from it.
+    Shards of 700 / 800 and of 128, 772, 101 (ragged), 499 tokens; grouped B/C; h0 != 0."""
+    import oracle
+    case = make_prefill(2, bounds[-1], 6, 64, 128, 3, 256, "bf16", h0_std=0.1, seed=51)
+    t = prefill_inputs(case)
+    W = len(bounds) - 1
+    sh = [slice(bounds[r], bounds[r + 1]) for r in range(W)]
+    cut = lambda a, s: a[:, s].contiguous()
+    loc = [ssd.prefill_local_state(cut(t["x"], s), cut(t["dt"], s), t["A"], cut(t["B"], s)) for s in sh]
+    h_all = torch.stack([l[0] for l in loc])
+    ld_all = torch.stack([l[1] for l in loc])
+    ys, hs = [], []
+    for r, s in enumerate(sh):
+        h_in = ssd.prefill_context_scan(r, h_all, ld_all, h0=t["h0"])
+        y, h = ssd.prefill(cut(t["x"], s), cut(t["dt"], s), t["A"], cut(t["B"], s), cut(t["C"], s), t["D"],
+                           chunk=256, h0=h_in)
+        ys.append(y)
+        hs.append(h)
+    torch.cuda.synchronize()
+    y_ref, hf_ref = oracle_subset(case, range(case.b), range(case.H))
+    check(_np(torch.cat(ys, 1)), y_ref, "bf16", "y")
+    check(_np(hs[-1]), hf_ref, "bf16", "h_final")
+    # the local state of one shard against the oracle from a zero state, and its log decay
+    s = sh[1]
+    _, h_loc_ref = oracle.ssd_recurrence(case.x[:, s], case.dt[:, s], case.A, case.B[:, s], case.C[:, s], case.D, None)
+    check(_np(h_all[1]), h_loc_ref, "bf16", "h_local")
+    ld_ref = (case.dt[:, s].astype(np.float64) * case.A.astype(np.float64)).sum(axis=1)
+    np.testing.assert_allclose(_np(ld_all[1]), ld_ref, rtol=1e-4)
