@@ -192,6 +192,12 @@ SSD_API int ssd_debug_starve_next_prefill(unsigned long long wait_limit_ns);
  * Errors: SSD_ERR_INVALID_ARG if nseg < 0. */
 SSD_API int ssd_debug_force_prefill_segments(int nseg);
 
+/* The same hook with the whole-unit count too: the first n_full (sequence, head) units (in
+ * order b * H + h) run in one pass and every later unit is split into nseg segments (the
+ * cost model's "ragged last wave" split).  n_full is clamped to b * H; nseg = 0 restores
+ * the cost model.  Errors: SSD_ERR_INVALID_ARG if n_full < 0 or nseg < 0. */
+SSD_API int ssd_debug_force_prefill_split(int n_full, int nseg);
+
 /* Decay-precision ablation for the tensor-core prefill ([CF-SSD] "Precision management":
  * decay parameters held in log space in fp32 and exponentiated at compute time; bf16 for
  * the decay exponentiation alone shifts the output).  mode 0 (the default) keeps every

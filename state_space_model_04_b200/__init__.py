@@ -13,6 +13,7 @@ from .ssd import (  # noqa: F401
     SSDError,
     debug_decay_precision,
     debug_force_prefill_segments,
+    debug_force_prefill_split,
     debug_starve_next_prefill,
     decode_loop,
     decode_step,

@@ -29,6 +29,7 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
 int prefill_tc_status(void* ws, cudaStream_t s);
 void prefill_tc_starve_next(unsigned long long wait_ns);
 void prefill_tc_force_segments(int nseg);
+void prefill_tc_force_split(int n_full, int nseg);
 void prefill_tc_decay_mode(int mode);
 int prefill_tc_segments(int b, int T, int H);
 size_t prefill_tc_local_state_workspace_bytes(int b, int T, int H);
@@ -300,6 +301,13 @@ int ssd_debug_decay_precision(int mode) {
     g_detail[0] = 0;
     if (mode < 0 || mode > 2) return set_error(SSD_ERR_INVALID_ARG, "decay precision mode %d is not 0, 1 or 2", mode);
     prefill_tc_decay_mode(mode);
+    return SSD_OK;
+}
+
+int ssd_debug_force_prefill_split(int n_full, int nseg) {
+    g_detail[0] = 0;
+    if (n_full < 0 || nseg < 0) return set_error(SSD_ERR_INVALID_ARG, "n_full %d / nseg %d negative", n_full, nseg);
+    prefill_tc_force_split(n_full, nseg);
     return SSD_OK;
 }
 

@@ -121,10 +121,14 @@ struct TcParams {
     __nv_bfloat16* y;
     int* status;
     int T, H, G;
-    int tseg, nseg;              // tokens per segment (a multiple of kBlk) and segments per sequence
-    float* seg_state;            // [b][H][nseg-1][P][N] fp32: a segment's local end state, then
+    // Work split.  A unit is one (sequence, head), u = bi * H + hd.  Units [0, n_full) run
+    // whole; each later unit ("split unit" su = u - n_full) is cut into nseg segments of
+    // tseg tokens (a multiple of kBlk; the last may be shorter).  The fused kernel's CTAs
+    // walk n_full whole units, then the split units' segments in order.
+    int n_full, tseg, nseg;
+    float* seg_state;            // [su][nseg-1][P][N] fp32: a segment's local end state, then
                                  // (after the scan) the state entering the next segment
-    float* seg_logdecay;         // [b][H][nseg-1]: sum of dt*A over a segment
+    float* seg_logdecay;         // [su][nseg-1]: sum of dt*A over a segment
     unsigned long long wait_ns;  // limit of every bounded wait
     int starve;                  // failure-detection test: the producer issues no loads
 };
@@ -350,12 +354,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int hd = blockIdx.x, bi = blockIdx.y, seg = blockIdx.z;
     const int T = prm.T, H = prm.H;
+    // this CTA's work item: a whole unit, or one segment of a split unit
+    int u, seg, nseg_u;
+    if ((int)blockIdx.x < prm.n_full) {
+        u = blockIdx.x, seg = 0, nseg_u = 1;
+    } else {
+        const int t = blockIdx.x - prm.n_full;
+        u = prm.n_full + t / prm.nseg, seg = t % prm.nseg, nseg_u = prm.nseg;
+    }
+    const int hd = u % H, bi = u / H;
     const int g = hd / (H / prm.G);
-    // this CTA's tokens: [tb, tb + tseg) clipped to T, in blocks of kBlk
+    // this CTA's tokens: [tb, tb + span), in blocks of kBlk
     const int tb = seg * prm.tseg;
-    const int nblk = (min(prm.tseg, T - tb) + kBlk - 1) / kBlk;
+    const int nblk = ((nseg_u == 1 ? T : min(prm.tseg, T - tb)) + kBlk - 1) / kBlk;
 
     uint8_t* small = smem + kSmall;
     uint64_t* bars = reinterpret_cast<uint64_t*>(small);              // BAR_COUNT barriers
@@ -644,8 +656,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         float Hs[32];              // fp32 running state H[p0 + k][r]
         {
             // state entering the segment: h0 for the first, the scanned segment states after it
-            const float* h0 = seg > 0 ? prm.seg_state + (((size_t)bi * H + hd) * (prm.nseg - 1) + seg - 1) * kP * kN
-                              : prm.h0 ? prm.h0 + ((size_t)bi * H + hd) * kP * kN
+            const float* h0 = seg > 0 ? prm.seg_state + ((size_t)(u - prm.n_full) * (prm.nseg - 1) + seg - 1) * kP * kN
+                              : prm.h0 ? prm.h0 + (size_t)u * kP * kN
                                        : nullptr;
 #pragma unroll
             for (int k = 0; k < 32; ++k) Hs[k] = h0 ? h0[(size_t)(p0 + k) * kN + r] : 0.f;
@@ -748,7 +760,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             }
             cs_last_prev = cs_last;
         }
-        if (!stopped && live && !*s_abort && prm.hf && seg == prm.nseg - 1) {
+        if (!stopped && live && !*s_abort && prm.hf && seg == nseg_u - 1) {
             float* hf = prm.hf + ((size_t)bi * H + hd) * kP * kN;
 #pragma unroll
             for (int j = 0; j < 32; ++j) hf[(size_t)(p0 + j) * kN + r] = Hs[j];
@@ -810,8 +822,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
 ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int hd = blockIdx.x, bi = blockIdx.y, seg = blockIdx.z;
     const int T = prm.T, H = prm.H;
+    // this CTA: segment seg (not the last) of split unit su
+    const int su = blockIdx.x / (prm.nseg - 1), seg = blockIdx.x % (prm.nseg - 1);
+    const int u = prm.n_full + su;
+    const int hd = u % H, bi = u / H;
     const int g = hd / (H / prm.G);
     const int tb = seg * prm.tseg;
     const int nblk = (min(prm.tseg, T - tb) + kBlk - 1) / kBlk;
@@ -960,7 +975,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
             if (u < nblk) logsum += cs_last;
         }
         if (!stopped && live && !*s_abort) {
-            const size_t o = ((size_t)bi * H + hd) * (prm.nseg - 1) + seg;
+            const size_t o = (size_t)su * (prm.nseg - 1) + seg;
             float* dst = prm.seg_state + o * kP * kN;
 #pragma unroll
             for (int j = 0; j < 32; ++j) dst[(size_t)(p0 + j) * kN + r] = Hs[j];
@@ -982,11 +997,12 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
 // the segments, loading kScanBatch segments' worth before the dependent updates.
 constexpr int kScanSplit = 8, kScanThreads = 128, kScanPer = kP * kN / (kScanSplit * kScanThreads), kScanBatch = 4;
 __global__ void __launch_bounds__(kScanThreads) ssd_segment_scan_kernel(const float* h0, float* seg_state,
-                                                                         const float* seg_logdecay, int H, int nseg) {
-    const int hd = blockIdx.x, bi = blockIdx.y;
-    const size_t o = ((size_t)bi * H + hd) * (nseg - 1);
+                                                                         const float* seg_logdecay, int n_full,
+                                                                         int nseg) {
+    const int su = blockIdx.x;  // split unit
+    const size_t o = (size_t)su * (nseg - 1);
     const int e0 = blockIdx.z * (kP * kN / kScanSplit) + threadIdx.x;  // entries e0 + kScanThreads * k
-    const float* h0p = h0 ? h0 + ((size_t)bi * H + hd) * kP * kN : nullptr;
+    const float* h0p = h0 ? h0 + (size_t)(n_full + su) * kP * kN : nullptr;
     float run[kScanPer];
 #pragma unroll
     for (int k = 0; k < kScanPer; ++k) run[k] = h0p ? h0p[e0 + kScanThreads * k] : 0.f;
@@ -1100,63 +1116,79 @@ int sm_count() {
     return n;
 }
 
-// Segments per sequence.  One CTA walks a segment's blocks one after another, so the
-// fused pass costs about (blocks per CTA) x (waves of CTAs) block-times when the waves
-// are full and about (all blocks / SMs) when CTAs of a ragged last wave finish early;
-// the model takes the mean of the two; a CTA's start (TMEM allocation, first loads) costs
-// about two more block-times.  Splitting the sequence adds CTAs when b * H alone leaves
-// SMs idle, at the price of the state pass (two CTAs per SM, measured at about 0.7 of a
-// fused block-time per block), the scan (about 0.4 block-times per segment) and a fixed
-// cost for the two extra launches.  nseg = 1 wherever the split does not pay by 5 %.
+// How the fused pass splits its work.  One CTA walks a unit's (or a segment's) blocks
+// one after another, so the fused pass costs about (blocks per CTA) x (waves of CTAs)
+// block-times when the waves are full and about (all blocks / SMs) when CTAs of a ragged
+// last wave finish early; the model takes the mean of the two; a CTA's start (TMEM
+// allocation, first loads) costs about two more block-times.  Splitting units into
+// segments adds CTAs where b * H alone leaves SMs idle -- all units when b * H is below
+// the SM count, or only the units of a ragged last wave -- at the price of the state pass
+// (two CTAs per SM, measured at about 0.7 of a fused block-time per block), the scan
+// (about 0.4 block-times per segment) and a fixed cost for the two extra launches.  No
+// split wherever the split does not pay by 5 %.
+struct SplitPlan {
+    int n_full, nseg, tseg;  // see TcParams
+};
 constexpr double kStatePassPerBlock = 0.7;
 constexpr double kCtaStartBlocks = 2.0;
 constexpr double kScanPerSegment = 0.4;
 constexpr double kSplitFixedBlocks = 5.0;
-std::atomic<int> g_force_nseg{0};
+std::atomic<int> g_force_nseg{0};     // 0: cost model
+std::atomic<int> g_force_nfull{-1};   // -1: every unit split when nseg > 1
 std::atomic<int> g_decay_mode{0};
-void plan_segments(int b, int T, int H, int* nseg, int* tseg) {
+
+// mean of the wave and flow estimates for `ctas` CTAs of `len` block-times
+double pass_cost(double ctas, double len, double sms) {
+    if (ctas <= 0) return 0.0;
+    return 0.5 * (std::ceil(ctas / sms) * len + std::max(ctas * len / sms, len));
+}
+
+SplitPlan plan_split(int b, int T, int H) {
     const int nb = (T + kBlk - 1) / kBlk;
+    const int units = b * H;
+    SplitPlan none{units, 1, nb * kBlk};
+    auto with_segments = [&](int n_full, int n) {
+        const int bps = (nb + n - 1) / n;
+        return SplitPlan{n_full, (nb + bps - 1) / bps, bps * kBlk};
+    };
     if (const int f = g_force_nseg.load()) {
-        const int bps = (nb + std::min(f, nb) - 1) / std::min(f, nb);
-        *tseg = bps * kBlk;
-        *nseg = (nb + bps - 1) / bps;
-        return;
+        const int n = std::min(f, nb);
+        if (n <= 1) return none;
+        const int nf = g_force_nfull.load();
+        return with_segments(nf < 0 ? 0 : std::min(nf, units), n);
     }
     const double sms = sm_count();
-    const double units = (double)b * H;
-    double best = 0.0;
-    int best_bps = nb;
-    for (int bps = nb; bps >= 1; --bps) {
-        const int n = (nb + bps - 1) / bps;
-        if (bps < nb && (nb + bps) / (bps + 1) == n) continue;  // same segment count as a longer bps
-        const double len = bps + kCtaStartBlocks;
-        const double waves = std::ceil(units * n / sms) * len;
-        const double flow = std::max(units * n * len / sms, len);
-        double cost = 0.5 * (waves + flow);
-        if (n > 1)
-            cost += kStatePassPerBlock * std::ceil(units * (n - 1) / (2.0 * sms)) * len + kScanPerSegment * n +
+    const double whole = pass_cost(units, nb + kCtaStartBlocks, sms);
+    SplitPlan best = none;
+    double best_cost = whole;
+    // candidates: split every unit, or only the units past the last whole wave
+    const int full_waves = (units / (int)sms) * (int)sms;
+    for (const int n_full : {0, full_waves}) {
+        if (n_full >= units || (n_full == full_waves && n_full == 0 && full_waves != 0)) continue;
+        const double r = units - n_full;
+        for (int bps = nb - 1; bps >= 1; --bps) {
+            const int n = (nb + bps - 1) / bps;
+            if ((nb + bps) / (bps + 1) == n) continue;  // same segment count as a longer bps
+            const double len = bps + kCtaStartBlocks;
+            double cost = (n_full ? std::ceil(n_full / sms) * (nb + kCtaStartBlocks) : 0.0) + pass_cost(r * n, len, sms);
+            cost += kStatePassPerBlock * std::ceil(r * (n - 1) / (2.0 * sms)) * len + kScanPerSegment * n +
                     kSplitFixedBlocks;
-        if (bps == nb || cost < 0.95 * best) {
-            best = cost;
-            best_bps = bps;
+            if (cost < 0.95 * best_cost) {
+                best_cost = cost;
+                best = SplitPlan{n_full, n, bps * kBlk};
+            }
         }
     }
-    *tseg = best_bps * kBlk;
-    *nseg = (nb + best_bps - 1) / best_bps;
+    return best;
 }
 }  // namespace
 
-int prefill_tc_segments(int b, int T, int H) {
-    int nseg = 1, tseg = T;
-    plan_segments(b, T, H, &nseg, &tseg);
-    return nseg;
-}
+int prefill_tc_segments(int b, int T, int H) { return plan_split(b, T, H).nseg; }
 
 size_t prefill_tc_workspace_bytes(int b, int T, int H) {
-    int nseg = 1, tseg = T;
-    plan_segments(b, T, H, &nseg, &tseg);
-    if (nseg == 1) return kSegOffset;
-    const size_t units = (size_t)b * H * (nseg - 1);
+    const SplitPlan sp = plan_split(b, T, H);
+    if (sp.nseg == 1) return kSegOffset;
+    const size_t units = (size_t)(b * H - sp.n_full) * (sp.nseg - 1);
     return kSegOffset + align256(units * kP * kN * sizeof(float)) + align256(units * sizeof(float));
 }
 
@@ -1164,7 +1196,14 @@ namespace {
 std::atomic<unsigned long long> g_starve_ns{0};
 }
 void prefill_tc_starve_next(unsigned long long wait_ns) { g_starve_ns.store(wait_ns); }
-void prefill_tc_force_segments(int nseg) { g_force_nseg.store(nseg); }
+void prefill_tc_force_segments(int nseg) {
+    g_force_nfull.store(-1);
+    g_force_nseg.store(nseg);
+}
+void prefill_tc_force_split(int n_full, int nseg) {
+    g_force_nfull.store(n_full);
+    g_force_nseg.store(nseg);
+}
 void prefill_tc_decay_mode(int mode) { g_decay_mode.store(mode); }
 
 int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt, const DtMap& dtm, const float* A,
@@ -1194,8 +1233,12 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     prm.T = T;
     prm.H = H;
     prm.G = G;
-    plan_segments(b, T, H, &prm.nseg, &prm.tseg);
-    const size_t units = (size_t)b * H * (prm.nseg - 1);
+    const SplitPlan sp = plan_split(b, T, H);
+    prm.n_full = sp.n_full;
+    prm.nseg = sp.nseg;
+    prm.tseg = sp.tseg;
+    const int n_split = b * H - sp.n_full;
+    const size_t units = (size_t)n_split * (prm.nseg - 1);
     prm.seg_state = reinterpret_cast<float*>(static_cast<char*>(ws) + kSegOffset);
     prm.seg_logdecay = reinterpret_cast<float*>(static_cast<char*>(ws) + kSegOffset +
                                                 align256(units * kP * kN * sizeof(float)));
@@ -1208,20 +1251,20 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
         SSD_CUDA_TRY(cudaFuncSetAttribute(state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSSmemBytes));
         {
             LaunchScope ls("ssd_segment_state", s);
-            state<<<dim3(H, b, prm.nseg - 1), kSThreads, kSSmemBytes, s>>>(prm);
+            state<<<(unsigned)units, kSThreads, kSSmemBytes, s>>>(prm);
         }
         SSD_CUDA_TRY(cudaGetLastError());
         {
             LaunchScope ls("ssd_segment_scan", s);
-            ssd_segment_scan_kernel<<<dim3(H, b, kScanSplit), kScanThreads, 0, s>>>(h0, prm.seg_state, prm.seg_logdecay,
-                                                                                    H, prm.nseg);
+            ssd_segment_scan_kernel<<<dim3(n_split, 1, kScanSplit), kScanThreads, 0, s>>>(
+                h0, prm.seg_state, prm.seg_logdecay, prm.n_full, prm.nseg);
         }
         SSD_CUDA_TRY(cudaGetLastError());
     }
     SSD_CUDA_TRY(cudaFuncSetAttribute(fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes));
     {
         LaunchScope ls("ssd_prefill_fused", s);
-        fused<<<dim3(H, b, prm.nseg), kThreads, kSmemBytes, s>>>(prm);
+        fused<<<(unsigned)(prm.n_full + (size_t)n_split * prm.nseg), kThreads, kSmemBytes, s>>>(prm);
     }
     SSD_CUDA_TRY(cudaGetLastError());
     return SSD_OK;
@@ -1262,6 +1305,7 @@ int launch_prefill_tc_local_state(int b, int T, int H, int G, const void* x, con
     const int nb = (T + kBlk - 1) / kBlk;
     prm.tseg = ((nb + n - 1) / n) * kBlk;
     const int pieces = (T + prm.tseg - 1) / prm.tseg;
+    prm.n_full = 0;
     prm.nseg = pieces + 1;  // the state pass writes pieces 0 .. nseg-2, i.e. every piece
     const size_t units = (size_t)b * H * pieces;
     prm.seg_state = reinterpret_cast<float*>(static_cast<char*>(ws) + kSegOffset);
@@ -1273,7 +1317,7 @@ int launch_prefill_tc_local_state(int b, int T, int H, int G, const void* x, con
                                       (int)kSSmemBytes));
     {
         LaunchScope ls("ssd_segment_state", s);
-        ssd_segment_state_kernel<0><<<dim3(H, b, pieces), kSThreads, kSSmemBytes, s>>>(prm);
+        ssd_segment_state_kernel<0><<<(unsigned)units, kSThreads, kSSmemBytes, s>>>(prm);
     }
     SSD_CUDA_TRY(cudaGetLastError());
     // piece q of unit u: state at (u * pieces + q) * P * N, log decay at u * pieces + q

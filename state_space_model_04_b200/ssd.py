@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill_segments.restype = _i
         L.ssd_debug_decay_precision.argtypes = [_i]
         L.ssd_debug_decay_precision.restype = _i
+        L.ssd_debug_force_prefill_split.argtypes = [_i, _i]
+        L.ssd_debug_force_prefill_split.restype = _i
         L.ssd_debug_force_prefill_segments.argtypes = [_i]
         L.ssd_debug_force_prefill_segments.restype = _i
         L.ssd_decode_workspace_size.argtypes = [_i] * 3
@@ -272,6 +274,12 @@ def debug_decay_precision(mode=0):
     """Decay-precision ablation of the tensor-core prefill: 0 fp32 (default), 1 exponentiated
     decay factors rounded to bf16, 2 log-space prefix sums rounded to bf16 before exp."""
     _check(lib().ssd_debug_decay_precision(int(mode)), "ssd_debug_decay_precision")
+
+
+def debug_force_prefill_split(n_full, nseg):
+    """Test hook: the first n_full (sequence, head) units run whole, the rest are split into
+    nseg segments (nseg = 0: the cost model)."""
+    _check(lib().ssd_debug_force_prefill_split(int(n_full), int(nseg)), "ssd_debug_force_prefill_split")
 
 
 def debug_force_prefill_segments(nseg=0):
