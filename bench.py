@@ -555,26 +555,30 @@ def decay_precision_ablation(ssd, torch, dev):
 
 
 def bench_prefill_configs(ssd, torch, dev, stream, args, clocks, barrier, max_over_ranks, world, pk, box):
-    """The other bf16 prefill configurations: the 130M-layer shape (b=1, T=4096, H=24) and
-    the long-context shape (b=1, T=65536, H=80, G=8), timed like the headline (inputs
-    resident, CUDA events on the launching stream, max over ranks).  On the fused path the
-    executed decomposition is the same for every requested chunk length, so one timing
-    serves L = 64, 128 and 256; TFLOP/s is given at each requested L and at the executed
-    128.  Both have few (sequence, head) pairs for 148 SMs, so the sequences are split into
-    segments (state pass + scan + fused pass); the segment count is reported."""
+    """The other prefill configurations: the tiny fp32 case (b=1, T=512, H=4, N=64; the fp32
+    four-kernel path, launch-latency bound), the 130M-layer shape (b=1, T=4096, H=24) and the
+    long-context shape (b=1, T=65536, H=80, G=8), timed like the headline (inputs resident,
+    CUDA events on the launching stream, max over ranks).  On the fused path the executed
+    decomposition is the same for every requested chunk length, so one timing serves
+    L = 64, 128 and 256; TFLOP/s is given at each requested L and for the decomposition that
+    ran.  The bf16 shapes have few (sequence, head) pairs for 148 SMs, so their sequences are
+    split into segments (state pass + scan + fused pass); the segment count is reported."""
     from ssd_inputs import make_config
     out = {}
-    for name, label in (("mamba2_130m_layer", "mamba2_130m_layer"), ("long_context_L256", "long_context")):
+    for name, label in (("tiny_f32", "tiny_f32"), ("mamba2_130m_layer", "mamba2_130m_layer"),
+                        ("long_context_L256", "long_context")):
         c = make_config(name)
+        io = ssd.SSD_F32 if c.dtype == "f32" else ssd.SSD_BF16
         b, T, H, P, N, G = c.b, c.T, c.H, c.P, c.N, c.G
-        def bf(bits):
+        def io_t(bits, vals):
+            if io == ssd.SSD_F32:
+                return torch.from_numpy(np.ascontiguousarray(vals, np.float32)).to(dev)
             return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
-        x, Bm, Cm = bf(c.x_bits), bf(c.B_bits), bf(c.C_bits)
+        x, Bm, Cm = io_t(c.x_bits, c.x), io_t(c.B_bits, c.B), io_t(c.C_bits, c.C)
         dt, A, D = (torch.from_numpy(v).to(dev) for v in (c.dt, c.A, c.D))
         y = torch.empty_like(x)
         hfin = torch.empty(b, H, P, N, device=dev)
-        ws = torch.empty(ssd.prefill_workspace_size(b, T, H, P, N, G, 256, ssd.SSD_BF16), dtype=torch.uint8,
-                         device=dev)
+        ws = torch.empty(ssd.prefill_workspace_size(b, T, H, P, N, G, 256, io), dtype=torch.uint8, device=dev)
         def step():
             ssd.prefill(x, dt, A, Bm, Cm, D, chunk=256, y=y, h_final=hfin, workspace=ws)
         for _ in range(args.warmup):
@@ -596,15 +600,17 @@ def bench_prefill_configs(ssd, torch, dev, stream, args, clocks, barrier, max_ov
         box[0] += ssd.launch_count() - n0
         barrier()
         ms = max_over_ranks(e0.elapsed_time(e1) / n_steps)
-        byt = prefill_bytes(b, T, H, P, N, G, with_h0=False)
+        byt = prefill_bytes(b, T, H, P, N, G, io_bytes=4 if io == ssd.SSD_F32 else 2, with_h0=False)
         gbs = byt * world / (ms * 1e-3) / 1e9
         entry = {"b": b, "T": T, "H": H, "G": G, "ms_per_step": ms, "tokens_per_s": job_rate(b * T, world, ms),
                  "bytes_per_step": byt, "hbm_gbs_alg": gbs, "hbm_frac": gbs / world / pk["hbm_gbs"],
-                 "tflops_executed_L128": job_rate(prefill_flops(b, T, H, P, N, G, EXEC_L_FUSED), world, ms) / 1e12,
+                 "dtype": c.dtype,
+                 "tflops_executed": job_rate(prefill_flops(b, T, H, P, N, G, EXEC_L_FUSED if io == ssd.SSD_BF16 else 256),
+                                             world, ms) / 1e12,
                  "tflops_at_requested_L": {str(L): job_rate(prefill_flops(b, T, H, P, N, G, L), world, ms) / 1e12
                                            for L in ((64, 128, 256) if label == "long_context" else (256,))},
                  "kernels": {k: {"launches": v[0] // n_steps, "avg_ms": v[1] / max(v[0], 1)} for k, v in kt.items()},
-                 "segments": ssd.prefill_segments(b, T, H, P, N, G, 256, ssd.SSD_BF16)}
+                 "segments": ssd.prefill_segments(b, T, H, P, N, G, 256, io)}
         out[label] = entry
         del x, Bm, Cm, dt, A, D, y, hfin, ws
         torch.cuda.empty_cache()
