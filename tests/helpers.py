@@ -3,8 +3,10 @@ sampled (sequence, head) subsets, and the tolerance metrics.
 
 Tolerances ("Compiler-First State Space Duality ..." validates fp32 against a reference
 at float32 rounding scale; the bf16 bar normalises by the largest output):
-  fp32 inputs : max_i |d_i| / max(|ref_i|, 1e-3 * max|ref|) <= 1e-4   (element-wise with a
-                floor so outputs that cancel to ~0 do not dominate)
+  fp32 inputs : max_i |d_i| / max(|ref_i|, 1e-2 * max|ref|) <= 1e-4   (element-wise with a
+                floor: each output is a sum of products whose terms reach max|ref|, so an
+                output that cancels to ~0 still carries an absolute rounding error of a few
+                fp32 ulps of max|ref|; the floor allows 1e-6 * max|ref|, about 8 ulps, there)
   bf16 inputs : max |d| / max |ref| <= 2e-2
 The same metrics apply to y and to the final / decode state.
 """
@@ -14,6 +16,7 @@ import torch
 import oracle
 
 TOL_F32 = 1e-4
+F32_FLOOR = 1e-2
 TOL_BF16 = 2e-2
 
 
@@ -23,7 +26,7 @@ def rel_max(got, ref):
     return float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30))
 
 
-def rel_floor(got, ref, floor=1e-3):
+def rel_floor(got, ref, floor=F32_FLOOR):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     den = np.maximum(np.abs(ref), floor * np.abs(ref).max())

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from ssd_inputs import make_config, make_prefill
-from tests.helpers import TOL_F32, check, oracle_subset, prefill_inputs, rel_max, run_prefill
+from tests.helpers import check, oracle_subset, prefill_inputs, rel_max, run_prefill
 
 pytestmark = pytest.mark.gpu
 
@@ -293,17 +293,10 @@ def test_dt_raw_matches_oracle(dtype, shape, nseg):
     dt_ref = oracle.dt_from_raw(raw, bias, lo, hi)
     assert (dt_ref == hi).any() and (dt_ref == lo).any()  # both ends of the clamp are exercised
     y_ref, hf_ref = oracle.ssd_recurrence(case.x, dt_ref, case.A, case.B, case.C, case.D, case.h0)
-    if dtype == "f32":
-        # The kernels form dt in fp32 (softplus within ~2 ulp) while the oracle forms it in
-        # fp64, so the two runs see step sizes that differ by that rounding; near zero
-        # crossings of y the element-wise metric with its 1e-3 floor magnifies it.  The gate
-        # here is the max-normalised fp32 bound.
-        for got, ref, what in ((_np(y), y_ref, "y"), (_np(hf), hf_ref, "h_final")):
-            e = rel_max(got, ref)
-            assert e <= TOL_F32, "%s: fp32 max-normalised error %.3e" % (what, e)
-    else:
-        check(_np(y), y_ref, dtype, "y")
-        check(_np(hf), hf_ref, dtype, "h_final")
+    # the kernels form dt in fp32 (softplus within ~2 ulp), the oracle in fp64: rounding
+    # the common fp32 metric covers
+    check(_np(y), y_ref, dtype, "y")
+    check(_np(hf), hf_ref, dtype, "h_final")
 
 
 def test_dt_raw_equals_preprocessed_dt():
