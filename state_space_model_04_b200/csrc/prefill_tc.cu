@@ -798,24 +798,33 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 
 // ------------------------------------------------------------------ segment state pass
 // For a sequence split into segments, the state a segment leaves behind when it starts
-// from zero ("Chunked recurrence" run over the segment alone): H_loc = sum over its blocks
-// of the decayed block states B^T (w o X), and the segment's total log decay sum(dt*A).
-// A scan over segments then gives every segment its entering state.  Only the state
-// recurrence runs here: one CTA per (head, sequence, segment), two CTAs per SM.
+// from zero ("Chunked recurrence" run over the segment alone) and the segment's total log
+// decay sum(dt*A).  A scan over segments then gives every segment its entering state.
+// One CTA per (head, sequence, segment), two CTAs per SM.
+//
+// The local state is the decayed sum over the segment's tokens,
+//   H_loc = sum_j exp(cs_end - cs_j) dt_j x_j B_j^T,
+// which the kernel evaluates as ONE tcgen05 accumulation over the whole segment: each
+// block's tokens are weighted straight to the segment end, so no state is carried,
+// rescaled or read back block by block.  Blocks are walked from the last to the first so
+// that the log decay from a block's end to the segment's end (`later`, the sum of the
+// totals of the blocks already walked) is known when the block arrives.  The weights
+// underflow only where exp(cs_end - cs_j) itself underflows fp32, as in the block-by-block
+// recurrence.
 //
 //   warp 0       TMA producer: B (two 64-column boxes) and X of a block into ring slot
-//                u & 1, two blocks ahead
-//   warp 1       TMEM owner and MMA issuer: S(u)^T = B^T (w o X) into TMEM buffer u & 1;
-//                its completion frees the slot
-//   warps 2-9    state group: block prefix sums, w o X in place over X in the slot,
-//                H <- exp(cs_last) H + S in registers
+//                u & 1, two blocks ahead (u counts blocks in walking order)
+//   warp 1       TMEM owner and MMA issuer: S^T += B^T (w o X); each block's completion
+//                frees its slot
+//   warps 2-9    state group: block prefix sums, w o X in place over X in the slot; at the
+//                end S^T out of TMEM to the segment-state buffer
 constexpr int kSThreads = 64 + kGroupThreads;
 constexpr uint32_t kSSlot = 3 * kRegion;             // B (n 0..63, 64..127), then X
 constexpr uint32_t kSX = 2 * kRegion;
 constexpr uint32_t kSSmall = 2 * kSSlot;
 constexpr uint32_t kSSmemBytes = kSSmall + 1024;
-constexpr uint32_t kSTmemCols = 128;                 // two 64-column S buffers
-enum { SB_FULL = 0, SB_EMPTY = 2, SB_XS = 4, SB_ACC = 6, SB_SFREE = 8, SB_DONE = 10, SB_COUNT };
+constexpr uint32_t kSTmemCols = 64;                  // one fp32 S^T accumulator (128 n x 64 p)
+enum { SB_FULL = 0, SB_EMPTY = 2, SB_XS = 4, SB_ACC = 6, SB_DONE = 7, SB_COUNT };
 
 template <int kDecay>
 __global__ void __launch_bounds__(kSThreads, 2)
@@ -825,11 +834,13 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
     const int T = prm.T, H = prm.H;
     // this CTA: segment seg (not the last) of split unit su
     const int su = blockIdx.x / (prm.nseg - 1), seg = blockIdx.x % (prm.nseg - 1);
-    const int u = prm.n_full + su;
-    const int hd = u % H, bi = u / H;
+    const int u0 = prm.n_full + su;
+    const int hd = u0 % H, bi = u0 / H;
     const int g = hd / (H / prm.G);
     const int tb = seg * prm.tseg;
     const int nblk = (min(prm.tseg, T - tb) + kBlk - 1) / kBlk;
+    // token offset of the u-th block walked (last block first)
+    auto block_t0 = [&](int u) { return tb + (nblk - 1 - u) * kBlk; };
 
     uint8_t* small = smem + kSSmall;
     uint64_t* bars = reinterpret_cast<uint64_t*>(small);
@@ -843,8 +854,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
     if (threadIdx.x == 0) {
         const bool misaligned = (sbase & 1023u) != 0;
         if (misaligned) atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (2 << 8));
-        for (int i = 0; i < SB_COUNT; ++i)
-            mbar_init(bar(i), (i == SB_XS || i == SB_XS + 1 || i == SB_SFREE || i == SB_SFREE + 1) ? kGroupThreads : 1);
+        for (int i = 0; i < SB_COUNT; ++i) mbar_init(bar(i), (i == SB_XS || i == SB_XS + 1) ? kGroupThreads : 1);
         *s_abort = misaligned ? 1 : 0;
         s_wait_ns = prm.wait_ns;
         s_ystop[0] = s_ystop[1] = 0;
@@ -865,11 +875,11 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
         if (lane == 0 && !*s_abort && !prm.starve) {
             int issued = 0;
             for (int u = 0; u < nblk; ++u) {
-                // slot u & 1 is free once S(u-2) has read it
+                // slot u & 1 is free once the MMAs of block u-2 have read it
                 if (u >= 2 && !mbar_wait(bar(SB_EMPTY + (u & 1)), ((u - 2) >> 1) & 1, s_abort, prm.status, 40)) break;
                 const uint32_t f = bar(SB_FULL + (u & 1));
                 const uint32_t slot = sbase + (u & 1) * kSSlot;
-                const int t0 = tb + u * kBlk;
+                const int t0 = block_t0(u);
                 mbar_expect_tx(f, 3 * kRegion);
                 tma_load_4d(slot, &prm.tm_B, f, 0, g, t0, bi);
                 tma_load_4d(slot + kRegion, &prm.tm_B, f, 64, g, t0, bi);
@@ -886,44 +896,38 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
             return warp_wait(bar(b), parity, s_abort, prm.status, where);
         };
         bool ok = __all_sync(0xffffffffu, !*s_abort);
-        if (ok) {
-            for (int u = 0; u < nblk && ok; ++u) {
-                // S buffer u & 1 was last read by the state group for block u - 2
-                ok = wt(SB_FULL + (u & 1), (u >> 1) & 1, 41) && wt(SB_XS + (u & 1), (u >> 1) & 1, 42) &&
-                     (u < 2 || wt(SB_SFREE + (u & 1), ((u - 2) >> 1) & 1, 43));
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t slot = sbase + (u & 1) * kSSlot;
-                const uint64_t dBt = sdesc(slot, kRegion, 1024), dXs = sdesc(slot + kSX, kRegion, 1024);
+        for (int u = 0; u < nblk && ok; ++u) {
+            ok = wt(SB_FULL + (u & 1), (u >> 1) & 1, 41) && wt(SB_XS + (u & 1), (u >> 1) & 1, 42);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t slot = sbase + (u & 1) * kSSlot;
+            const uint64_t dBt = sdesc(slot, kRegion, 1024), dXs = sdesc(slot + kSX, kRegion, 1024);
 #pragma unroll
-                for (int kk = 0; kk < kBlk / 16; ++kk)
-                    mma_ss_w(tmem + (u & 1) * 64, dBt + kk * 128, dXs + kk * 128, id_s, kk > 0);
-                mma_commit_w(bar(SB_ACC + (u & 1)));
-                mma_commit_w(bar(SB_EMPTY + (u & 1)));
-            }
-            mma_commit_w(bar(SB_DONE));
-            mbar_drain(bar(SB_DONE), 0);
+            for (int kk = 0; kk < kBlk / 16; ++kk)
+                mma_ss_w(tmem, dBt + kk * 128, dXs + kk * 128, id_s, (u > 0 || kk > 0) ? 1u : 0u);
+            mma_commit_w(bar(SB_EMPTY + (u & 1)));
         }
+        // the accumulator is complete (or, on the abort path, abandoned) once every MMA issued
+        // above has landed; the drain keeps the TMEM alive until then
+        mma_commit_w(bar(SB_ACC));
+        mma_commit_w(bar(SB_DONE));
+        mbar_drain(bar(SB_DONE), 0);
     } else {
         // ================================================================ state group
         const int q = warp & 3, half = (warp - 2) >> 2;
-        const int r = q * 32 + lane;  // token row of a block (w o X) and state row n (S, H)
+        const int r = q * 32 + lane;  // token row of a block (w o X) and state row n (S)
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
         const int p0 = half * 32;
         const float Ah = prm.A[hd];
-        float Hs[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) Hs[k] = 0.f;
         auto load_dt = [&](int u) {
-            const int tok = tb + u * kBlk + r;
+            const int tok = block_t0(u) + r;
             return (u < nblk && tok < T) ? dt_value(__ldg(prm.dt + ((size_t)bi * T + tok) * H + hd), prm.dtm, hd) : 0.f;
         };
         bool live = __all_sync(0xffffffffu, !*s_abort);
         bool stopped = false;
         float dt_a = load_dt(0), dt_b = load_dt(1);
-        float cs_last_prev = 0.f, logsum = 0.f;
-        // iteration u: w o X of block u, then the state update with S(u-1)
-        for (int u = 0; u <= nblk; ++u) {
+        float later = 0.f;  // log decay from the end of the current block to the end of the segment
+        for (int u = 0; u < nblk; ++u) {
             const int s = u & 1;
             const float dtv = dt_a;
             dt_a = dt_b;
@@ -937,11 +941,12 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
                 stopped = true;
                 break;
             }
-            if (live && u < nblk) {
+            if (live) {
                 live = warp_wait(bar(SB_FULL + s), (u >> 1) & 1, s_abort, prm.status, 44);
                 if (live) {
-                    // w_j x_j in place, one packed bf16x2 multiply per element pair
-                    const __nv_bfloat162 w2 = __float2bfloat162_rn(dexp<kDecay>(__expf(cs_last - cs)) * dtv);
+                    // w_j x_j in place with w_j = exp(cs_end - cs_j) dt_j, one packed bf16x2
+                    // multiply per element pair
+                    const __nv_bfloat162 w2 = __float2bfloat162_rn(dexp<kDecay>(__expf(later + cs_last - cs)) * dtv);
                     uint8_t* xs = smem + s * kSSlot + kSX;
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
@@ -955,31 +960,23 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
                     mbar_arrive(bar(SB_XS + s));
                 }
             }
-            if (live && u >= 1) {
-                // H <- exp(cs_last(u-1)) H + S(u-1)
-                const int sp = (u - 1) & 1;
-                live = warp_wait(bar(SB_ACC + sp), ((u - 1) >> 1) & 1, s_abort, prm.status, 45);
-                if (live) {
-                    tc_fence_after();
-                    uint32_t raw[32];
-                    SSD_TMEM_LD32(tmem + lane_addr + sp * 64 + p0, raw);
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    mbar_arrive(bar(SB_SFREE + sp));
-                    const float gam = dexp<kDecay>(__expf(cs_last_prev));
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) Hs[j] = fmaf(gam, Hs[j], __uint_as_float(raw[j]));
-                }
-            }
-            cs_last_prev = cs_last;
-            if (u < nblk) logsum += cs_last;
+            later += cs_last;
         }
-        if (!stopped && live && !*s_abort) {
-            const size_t o = (size_t)su * (prm.nseg - 1) + seg;
-            float* dst = prm.seg_state + o * kP * kN;
+        // H_loc^T row n = r, columns [p0, p0 + 32) out of the accumulator
+        if (!stopped && live) live = warp_wait(bar(SB_ACC), 0, s_abort, prm.status, 45);
+        if (!stopped && live) {
+            tc_fence_after();
+            uint32_t raw[32];
+            SSD_TMEM_LD32(tmem + lane_addr + p0, raw);
+            tmem_wait_ld();
+            tc_fence_before();
+            if (!*s_abort) {
+                const size_t o = (size_t)su * (prm.nseg - 1) + seg;
+                float* dst = prm.seg_state + o * kP * kN;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dst[(size_t)(p0 + j) * kN + r] = Hs[j];
-            if (r == 0 && half == 0) prm.seg_logdecay[o] = logsum;
+                for (int j = 0; j < 32; ++j) dst[(size_t)(p0 + j) * kN + r] = __uint_as_float(raw[j]);
+                if (r == 0 && half == 0) prm.seg_logdecay[o] = later;
+            }
         }
     }
 
