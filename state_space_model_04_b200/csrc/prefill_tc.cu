@@ -800,7 +800,9 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 // For a sequence split into segments, the state a segment leaves behind when it starts
 // from zero ("Chunked recurrence" run over the segment alone) and the segment's total log
 // decay sum(dt*A).  A scan over segments then gives every segment its entering state.
-// One CTA per (head, sequence, segment), two CTAs per SM.
+// One CTA per segment of kHP heads of one sequence that share a B/C group: with kHP = 2 the
+// group's B tile is loaded once for both heads and one MMA (N = 128) serves both, which cuts
+// the bytes a block moves from 48 KB per head to 32 KB.
 //
 // The local state is the decayed sum over the segment's tokens,
 //   H_loc = sum_j exp(cs_end - cs_j) dt_j x_j B_j^T,
@@ -812,39 +814,48 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 // underflow only where exp(cs_end - cs_j) itself underflows fp32, as in the block-by-block
 // recurrence.
 //
-//   warp 0       TMA producer: B (two 64-column boxes) and X of a block into ring slot
-//                u & 1, two blocks ahead (u counts blocks in walking order)
-//   warp 1       TMEM owner and MMA issuer: S^T += B^T (w o X); each block's completion
-//                frees its slot
-//   warps 2-9    state group: block prefix sums, w o X in place over X in the slot; at the
-//                end S^T out of TMEM to the segment-state buffer
+//   warp 0       TMA producer: B (two 64-column boxes) and the X of each head of a block
+//                into ring slot u % kSlots (u counts blocks in walking order)
+//   warp 1       TMEM owner and MMA issuer: S^T += B^T (w o X), N = 64 kHP (the heads' X
+//                tiles side by side); each block's completion frees its slot
+//   warps 2-9    state group: block prefix sums, w o X in place over X in the slot (one
+//                head per half of the group when kHP = 2); at the end S^T out of TMEM to
+//                the segment-state buffer
 constexpr int kSThreads = 64 + kGroupThreads;
-constexpr uint32_t kSSlot = 3 * kRegion;             // B (n 0..63, 64..127), then X
-constexpr uint32_t kSX = 2 * kRegion;
-constexpr uint32_t kSSmall = 2 * kSSlot;
-constexpr uint32_t kSSmemBytes = kSSmall + 1024;
-constexpr uint32_t kSTmemCols = 64;                  // one fp32 S^T accumulator (128 n x 64 p)
-enum { SB_FULL = 0, SB_EMPTY = 2, SB_XS = 4, SB_ACC = 6, SB_DONE = 7, SB_COUNT };
+constexpr uint32_t kSX = 2 * kRegion;                // X tiles follow the two B regions
+template <int kHP>
+struct SPass {
+    static constexpr uint32_t kSlot = (2 + kHP) * kRegion;  // B (n 0..63, 64..127), then X per head
+    static constexpr int kSlots = kHP == 1 ? 2 : 3;          // 96 KB or 192 KB of loads in flight
+    static constexpr uint32_t kSmall = kSlots * kSlot;
+    static constexpr uint32_t kSmem = kSmall + 1024;
+    static constexpr uint32_t kTmemCols = 64 * kHP;          // fp32 S^T accumulators (128 n x 64 p each)
+    static constexpr int kMinBlocks = kHP == 1 ? 2 : 1;      // CTAs per SM
+};
+static_assert(SPass<1>::kSmem * 2 <= 232448 && SPass<2>::kSmem <= 232448, "state pass shared memory");
+enum { SB_FULL = 0, SB_EMPTY = 3, SB_XS = 6, SB_ACC = 9, SB_DONE = 10, SB_COUNT };
 
-template <int kDecay>
-__global__ void __launch_bounds__(kSThreads, 2)
+template <int kDecay, int kHP>
+__global__ void __launch_bounds__(kSThreads, SPass<kHP>::kMinBlocks)
 ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
+    using SP = SPass<kHP>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = prm.T, H = prm.H;
-    // this CTA: segment seg (not the last) of split unit su
-    const int su = blockIdx.x / (prm.nseg - 1), seg = blockIdx.x % (prm.nseg - 1);
-    const int u0 = prm.n_full + su;
-    const int hd = u0 % H, bi = u0 / H;
-    const int g = hd / (H / prm.G);
+    // this CTA: segment seg (not the last) of split units su0 .. su0 + kHP - 1 (heads
+    // hd0 .. hd0 + kHP - 1 of one sequence, in one group)
+    const int su0 = (blockIdx.x / (prm.nseg - 1)) * kHP, seg = blockIdx.x % (prm.nseg - 1);
+    const int u0 = prm.n_full + su0;
+    const int hd0 = u0 % H, bi = u0 / H;
+    const int g = hd0 / (H / prm.G);
     const int tb = seg * prm.tseg;
     const int nblk = (min(prm.tseg, T - tb) + kBlk - 1) / kBlk;
     // token offset of the u-th block walked (last block first)
     auto block_t0 = [&](int u) { return tb + (nblk - 1 - u) * kBlk; };
 
-    uint8_t* small = smem + kSSmall;
+    uint8_t* small = smem + SP::kSmall;
     uint64_t* bars = reinterpret_cast<uint64_t*>(small);
-    float* s_tot = reinterpret_cast<float*>(small + 128);          // [2][4] quadrant sums
+    float* s_tot = reinterpret_cast<float*>(small + 128);          // [2][kHP][4] quadrant sums
     volatile int* s_abort = reinterpret_cast<volatile int*>(small + 192);
     volatile int* s_ystop = s_abort + 1;                           // [2]
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(small + 208);
@@ -854,7 +865,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
     if (threadIdx.x == 0) {
         const bool misaligned = (sbase & 1023u) != 0;
         if (misaligned) atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (2 << 8));
-        for (int i = 0; i < SB_COUNT; ++i) mbar_init(bar(i), (i == SB_XS || i == SB_XS + 1) ? kGroupThreads : 1);
+        for (int i = 0; i < SB_COUNT; ++i) mbar_init(bar(i), (i >= SB_XS && i < SB_XS + 3) ? kGroupThreads : 1);
         *s_abort = misaligned ? 1 : 0;
         s_wait_ns = prm.wait_ns;
         s_ystop[0] = s_ystop[1] = 0;
@@ -862,50 +873,53 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
-                     "r"(kSTmemCols));
+                     "r"(SP::kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    constexpr int kS = SP::kSlots;
 
     if (warp == 0) {
         // ================================================================ TMA producer
         if (lane == 0 && !*s_abort && !prm.starve) {
             int issued = 0;
             for (int u = 0; u < nblk; ++u) {
-                // slot u & 1 is free once the MMAs of block u-2 have read it
-                if (u >= 2 && !mbar_wait(bar(SB_EMPTY + (u & 1)), ((u - 2) >> 1) & 1, s_abort, prm.status, 40)) break;
-                const uint32_t f = bar(SB_FULL + (u & 1));
-                const uint32_t slot = sbase + (u & 1) * kSSlot;
+                // slot u % kS is free once the MMAs of block u - kS have read it
+                if (u >= kS && !mbar_wait(bar(SB_EMPTY + u % kS), ((u - kS) / kS) & 1, s_abort, prm.status, 40)) break;
+                const uint32_t f = bar(SB_FULL + u % kS);
+                const uint32_t slot = sbase + (u % kS) * SP::kSlot;
                 const int t0 = block_t0(u);
-                mbar_expect_tx(f, 3 * kRegion);
+                mbar_expect_tx(f, (2 + kHP) * kRegion);
                 tma_load_4d(slot, &prm.tm_B, f, 0, g, t0, bi);
                 tma_load_4d(slot + kRegion, &prm.tm_B, f, 64, g, t0, bi);
-                tma_load_4d(slot + kSX, &prm.tm_x, f, 0, hd, t0, bi);
+#pragma unroll
+                for (int h = 0; h < kHP; ++h) tma_load_4d(slot + kSX + h * kRegion, &prm.tm_x, f, 0, hd0 + h, t0, bi);
                 issued = u + 1;
             }
-            for (int u = issued - 2; u < issued; ++u)
-                if (u >= 0) mbar_drain(bar(SB_FULL + (u & 1)), (u >> 1) & 1);
+            for (int u = issued - kS; u < issued; ++u)
+                if (u >= 0) mbar_drain(bar(SB_FULL + u % kS), (u / kS) & 1);
         }
     } else if (warp == 1) {
         // ================================================================ MMA issuer
-        constexpr uint32_t id_s = idesc_bf16(128, 64, 1, 1);  // A B^T (MN-major), B w o X (MN-major)
+        // A B^T (MN-major), B the heads' w o X tiles (MN-major, 64-column atoms a region apart)
+        constexpr uint32_t id_s = idesc_bf16(128, 64 * kHP, 1, 1);
         auto wt = [&](int b, uint32_t parity, int where) {
             return warp_wait(bar(b), parity, s_abort, prm.status, where);
         };
         bool ok = __all_sync(0xffffffffu, !*s_abort);
         for (int u = 0; u < nblk && ok; ++u) {
-            ok = wt(SB_FULL + (u & 1), (u >> 1) & 1, 41) && wt(SB_XS + (u & 1), (u >> 1) & 1, 42);
+            ok = wt(SB_FULL + u % kS, (u / kS) & 1, 41) && wt(SB_XS + u % kS, (u / kS) & 1, 42);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t slot = sbase + (u & 1) * kSSlot;
+            const uint32_t slot = sbase + (u % kS) * SP::kSlot;
             const uint64_t dBt = sdesc(slot, kRegion, 1024), dXs = sdesc(slot + kSX, kRegion, 1024);
 #pragma unroll
             for (int kk = 0; kk < kBlk / 16; ++kk)
                 mma_ss_w(tmem, dBt + kk * 128, dXs + kk * 128, id_s, (u > 0 || kk > 0) ? 1u : 0u);
-            mma_commit_w(bar(SB_EMPTY + (u & 1)));
+            mma_commit_w(bar(SB_EMPTY + u % kS));
         }
         // the accumulator is complete (or, on the abort path, abandoned) once every MMA issued
         // above has landed; the drain keeps the TMEM alive until then
@@ -917,7 +931,12 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
         const int q = warp & 3, half = (warp - 2) >> 2;
         const int r = q * 32 + lane;  // token row of a block (w o X) and state row n (S)
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-        const int p0 = half * 32;
+        // kHP = 1: both halves on the one head, 32 of its 64 p columns each;
+        // kHP = 2: half h takes head hd0 + h, all 64 columns
+        const int h = kHP == 2 ? half : 0;
+        const int hd = hd0 + h;
+        constexpr int kChunks = 8 / (3 - kHP);  // 16-byte chunks of an X row per thread: 4 or 8
+        const int c0 = kHP == 2 ? 0 : half * 4;
         const float Ah = prm.A[hd];
         auto load_dt = [&](int u) {
             const int tok = block_t0(u) + r;
@@ -928,13 +947,14 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
         float dt_a = load_dt(0), dt_b = load_dt(1);
         float later = 0.f;  // log decay from the end of the current block to the end of the segment
         for (int u = 0; u < nblk; ++u) {
-            const int s = u & 1;
+            const int s = u & 1;  // stop-flag and quadrant-sum buffer
             const float dtv = dt_a;
             dt_a = dt_b;
             dt_b = load_dt(u + 2);
             if (!live || *s_abort) s_ystop[s] = 1;
             float cend[4], cs_last;
-            float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_tot + s * 4, 4, cs_last, cend);
+            float cs = block_cumsum(dtv * Ah, q, lane, kHP == 2 || half == 0, s_tot + (s * kHP + h) * 4, 4, cs_last,
+                                    cend);
             cs = dlog<kDecay>(cs);
             cs_last = dlog<kDecay>(cs_last);
             if (s_ystop[s]) {
@@ -942,40 +962,46 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
                 break;
             }
             if (live) {
-                live = warp_wait(bar(SB_FULL + s), (u >> 1) & 1, s_abort, prm.status, 44);
+                live = warp_wait(bar(SB_FULL + u % kS), (u / kS) & 1, s_abort, prm.status, 44);
                 if (live) {
                     // w_j x_j in place with w_j = exp(cs_end - cs_j) dt_j, one packed bf16x2
                     // multiply per element pair
                     const __nv_bfloat162 w2 = __float2bfloat162_rn(dexp<kDecay>(__expf(later + cs_last - cs)) * dtv);
-                    uint8_t* xs = smem + s * kSSlot + kSX;
+                    uint8_t* xs = smem + (u % kS) * SP::kSlot + kSX + h * kRegion;
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        uint4 uv = *reinterpret_cast<const uint4*>(xs + swz(r, half * 4 + c4));
+                    for (int c4 = 0; c4 < kChunks; ++c4) {
+                        uint4 uv = *reinterpret_cast<const uint4*>(xs + swz(r, c0 + c4));
                         __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&uv);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) e[j] = __hmul2(e[j], w2);
-                        *reinterpret_cast<uint4*>(xs + swz(r, half * 4 + c4)) = uv;
+                        *reinterpret_cast<uint4*>(xs + swz(r, c0 + c4)) = uv;
                     }
                     fence_proxy_async();
-                    mbar_arrive(bar(SB_XS + s));
+                    mbar_arrive(bar(SB_XS + u % kS));
                 }
             }
             later += cs_last;
         }
-        // H_loc^T row n = r, columns [p0, p0 + 32) out of the accumulator
+        // H_loc^T row n = r of head hd, this thread's p columns, out of the accumulator
         if (!stopped && live) live = warp_wait(bar(SB_ACC), 0, s_abort, prm.status, 45);
         if (!stopped && live) {
             tc_fence_after();
-            uint32_t raw[32];
-            SSD_TMEM_LD32(tmem + lane_addr + p0, raw);
+            constexpr int kCols = 32 * kHP;  // 32 (half of one head) or 64 (a whole head)
+            const int pbase = kHP == 2 ? 0 : half * 32;
+            uint32_t raw[kCols];
+            SSD_TMEM_LD32(tmem + lane_addr + h * 64 + pbase, raw);
+            if constexpr (kHP == 2) {
+                uint32_t* raw_hi = raw + 32;
+                SSD_TMEM_LD32(tmem + lane_addr + h * 64 + 32, raw_hi);
+            }
             tmem_wait_ld();
             tc_fence_before();
             if (!*s_abort) {
-                const size_t o = (size_t)su * (prm.nseg - 1) + seg;
+                const size_t o = (size_t)(su0 + h) * (prm.nseg - 1) + seg;
                 float* dst = prm.seg_state + o * kP * kN;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) dst[(size_t)(p0 + j) * kN + r] = __uint_as_float(raw[j]);
-                if (r == 0 && half == 0) prm.seg_logdecay[o] = later;
+                for (int j = 0; j < kCols; ++j) dst[(size_t)(pbase + j) * kN + r] = __uint_as_float(raw[j]);
+                if (r == 0 && (kHP == 2 || half == 0)) prm.seg_logdecay[o] = later;
             }
         }
     }
@@ -984,8 +1010,36 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kSTmemCols));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(SP::kTmemCols));
     }
+}
+
+int sm_count();
+
+// Launches the state pass over the split units [n_full, n_full + n_split): two heads per CTA
+// where both heads of every pair share a B/C group, one otherwise.
+template <int kHP>
+int launch_state_pass_hp(const TcParams& prm, int decay, unsigned grid, cudaStream_t s) {
+    auto k = decay == 1 ? ssd_segment_state_kernel<1, kHP>
+             : decay == 2 ? ssd_segment_state_kernel<2, kHP>
+                          : ssd_segment_state_kernel<0, kHP>;
+    SSD_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SPass<kHP>::kSmem));
+    {
+        LaunchScope ls("ssd_segment_state", s);
+        k<<<grid, kSThreads, SPass<kHP>::kSmem, s>>>(prm);
+    }
+    SSD_CUDA_TRY(cudaGetLastError());
+    return SSD_OK;
+}
+int launch_state_pass(const TcParams& prm, int n_split, int decay, cudaStream_t s) {
+    // a pair (u, u + 1) starts at an even head, so both heads sit in one group when the
+    // group size is even; the split units must then pair up exactly.  Pairs run one CTA per
+    // SM, so they are used only when their grid fills the GPU (else two single-head CTAs per
+    // SM spread the work wider).
+    const bool pair = (prm.H / prm.G) % 2 == 0 && prm.n_full % 2 == 0 && n_split % 2 == 0 &&
+                      (double)(n_split / 2) * (prm.nseg - 1) >= sm_count();
+    const unsigned grid = (unsigned)((size_t)(n_split / (pair ? 2 : 1)) * (prm.nseg - 1));
+    return pair ? launch_state_pass_hp<2>(prm, decay, grid, s) : launch_state_pass_hp<1>(prm, decay, grid, s);
 }
 
 // Entering state of every segment after the first, in place of the local states:
@@ -1126,7 +1180,7 @@ int sm_count() {
 struct SplitPlan {
     int n_full, nseg, tseg;  // see TcParams
 };
-constexpr double kStatePassPerBlock = 0.7;
+constexpr double kStatePassPerBlock = 0.7;  // single-head state pass; the paired one measures ~0.5
 constexpr double kCtaStartBlocks = 2.0;
 constexpr double kScanPerSegment = 0.4;
 constexpr double kSplitFixedBlocks = 5.0;
@@ -1219,8 +1273,6 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     const int decay = g_decay_mode.load();
     auto fused = decay == 1 ? ssd_prefill_fused_kernel<1> : decay == 2 ? ssd_prefill_fused_kernel<2>
                                                                         : ssd_prefill_fused_kernel<0>;
-    auto state = decay == 1 ? ssd_segment_state_kernel<1> : decay == 2 ? ssd_segment_state_kernel<2>
-                                                                        : ssd_segment_state_kernel<0>;
     prm.A = A;
     prm.D = D;
     prm.h0 = h0;
@@ -1245,12 +1297,7 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     SSD_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), s));
     if (prm.nseg > 1) {
         // local end states of all segments but the last, then their scan
-        SSD_CUDA_TRY(cudaFuncSetAttribute(state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSSmemBytes));
-        {
-            LaunchScope ls("ssd_segment_state", s);
-            state<<<(unsigned)units, kSThreads, kSSmemBytes, s>>>(prm);
-        }
-        SSD_CUDA_TRY(cudaGetLastError());
+        if ((st = launch_state_pass(prm, n_split, decay, s)) != SSD_OK) return st;
         {
             LaunchScope ls("ssd_segment_scan", s);
             ssd_segment_scan_kernel<<<dim3(n_split, 1, kScanSplit), kScanThreads, 0, s>>>(
@@ -1310,13 +1357,7 @@ int launch_prefill_tc_local_state(int b, int T, int H, int G, const void* x, con
                                                 align256(units * kP * kN * sizeof(float)));
     prm.wait_ns = kWaitLimitNs;
     SSD_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), s));
-    SSD_CUDA_TRY(cudaFuncSetAttribute(ssd_segment_state_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)kSSmemBytes));
-    {
-        LaunchScope ls("ssd_segment_state", s);
-        ssd_segment_state_kernel<0><<<(unsigned)units, kSThreads, kSSmemBytes, s>>>(prm);
-    }
-    SSD_CUDA_TRY(cudaGetLastError());
+    if ((st = launch_state_pass(prm, b * H, 0, s)) != SSD_OK) return st;
     // piece q of unit u: state at (u * pieces + q) * P * N, log decay at u * pieces + q
     {
         LaunchScope ls("ssd_state_fold", s);

@@ -150,6 +150,27 @@ def test_sequence_split_matches_oracle(nseg):
     check(_np(hf), _np(h1), "bf16", "h_final split vs one pass")
 
 
+def test_paired_state_pass_matches_oracle():
+    """The segment state pass runs two heads of one B/C group per CTA when the group size is
+    even and the pairs fill the GPU (here 16 pairs x 15 segments = 240 CTAs on 148 SMs): both
+    heads of a pair, and pairs at both ends of the head range, match the oracle and the
+    unsplit pass.  T = 4000 leaves a ragged last block."""
+    case = make_prefill(1, 4000, 32, 64, 128, 4, 256, "bf16", h0_std=0.1, seed=61)
+    ssd.debug_force_prefill_segments(1)
+    try:
+        y1, h1, _ = run_prefill(ssd, case)
+        ssd.debug_force_prefill_segments(16)
+        y, hf, _ = run_prefill(ssd, case)
+    finally:
+        ssd.debug_force_prefill_segments(0)
+    heads = [0, 1, 6, 7, 8, 9, 30, 31]
+    y_ref, hf_ref = oracle_subset(case, [0], heads)
+    check(_np(y)[:, :, heads], y_ref, "bf16", "y")
+    check(_np(hf)[:, heads], hf_ref, "bf16", "h_final")
+    check(_np(y), _np(y1), "bf16", "y split vs one pass")
+    check(_np(hf), _np(h1), "bf16", "h_final split vs one pass")
+
+
 def test_causality_bitwise():
     case = make_prefill(1, 768, 4, 64, 128, 1, 256, "bf16", seed=7)
     y, _, t = run_prefill(ssd, case)
