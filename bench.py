@@ -202,14 +202,26 @@ def job_rate(units_per_rank, world, ms_max):
 
 
 # ----------------------------------------------------------------------------- helpers
-def sha_prefix(path):
+def sha_prefix(path, upto=None):
+    """sha256[:12] of a source file, or of its text before the first line that starts with
+    `upto` (the part a kernel's code depends on, when later sections hold other kernels)."""
     with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:12]
+        data = f.read()
+    if upto:
+        i = data.find(b"\n" + upto.encode())
+        if i >= 0:
+            data = data[:i + 1]
+    return hashlib.sha256(data).hexdigest()[:12]
+
+
+# the fused prefill kernel and the helpers it uses end where the segment state pass begins
+KERNEL_SOURCE_END = {"ssd_prefill_fused": "// ------------------------------------------------------------------ segment state pass"}
 
 
 def dram_traffic(kernel):
-    """Per-launch DRAM bytes of `kernel` from profiles/dram_traffic.txt, only if the source
-    file recorded there is unchanged since the ncu capture (else None)."""
+    """Per-launch DRAM bytes of `kernel` from profiles/dram_traffic.txt, only if the kernel's
+    source (the file up to KERNEL_SOURCE_END, else the whole file) is unchanged since the ncu
+    capture (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -220,7 +232,7 @@ def dram_traffic(kernel):
         if len(parts) >= 4 and parts[0] == kernel:
             src, sha, per_launch = parts[1], parts[2], float(parts[3])
             full = os.path.join(ROOT, src)
-            if os.path.exists(full) and sha_prefix(full) == sha:
+            if os.path.exists(full) and sha_prefix(full, KERNEL_SOURCE_END.get(kernel)) == sha:
                 return per_launch
     return None
 

@@ -9,7 +9,9 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 #include <string>
+#include <tuple>
 #include <vector>
 
 namespace ssd {
@@ -63,6 +65,23 @@ int set_error(int status, const char* fmt, ...) {
 
 int cuda_status(cudaError_t e, const char* where) {
     return set_error(SSD_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// The dynamic shared-memory limit is a per-device attribute of a kernel: set it once per
+// (kernel, device, size) instead of on every launch (a host call each time).
+int smem_limit_once(const void* func, int bytes) {
+    static std::mutex mu;
+    static std::vector<std::tuple<const void*, int, int>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lock(mu);
+    for (const auto& d : done)
+        if (std::get<0>(d) == func && std::get<1>(d) == dev && std::get<2>(d) >= bytes) return SSD_OK;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(MaxDynamicSharedMemorySize)");
+    done.emplace_back(func, dev, bytes);
+    return SSD_OK;
 }
 
 // ---- launch accounting and event timing

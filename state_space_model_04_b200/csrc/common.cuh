@@ -50,6 +50,9 @@ __device__ __forceinline__ float dt_value(float v, const DtMap& m, int h) {
 // Map a CUDA error to a status with detail.
 int cuda_status(cudaError_t e, const char* where);
 
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current device, once.
+int smem_limit_once(const void* func, int bytes);
+
 // Launch accounting and optional per-kernel event timing (see ssd_profile_begin).
 void count_launches(uint64_t n);
 void prof_start(const char* name, cudaStream_t s);  // no-op unless profiling

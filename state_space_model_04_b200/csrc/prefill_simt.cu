@@ -312,7 +312,7 @@ int run(int b, int T, int H, int G, int L, const void* x, const float* dt, const
     }
     const size_t smem = sizeof(float) * (2 * 64 * (N + 1) + 64 * 65 + 64 * kP);
     auto k4 = chunk_output_kernel<IoT, CsT, N>;
-    SSD_CUDA_TRY(cudaFuncSetAttribute(k4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    if (const int st = smem_limit_once((const void*)k4, (int)smem)) return st;
     {
         LaunchScope ls("simt_chunk_output", s);
         k4<<<dim3(nc * ((L + 63) / 64), H, b), kThreads, smem, s>>>(T, H, G, L, nc, xi, dt, dtm, Bi, Ci, D, cs, S,

@@ -1023,7 +1023,7 @@ int launch_state_pass_hp(const TcParams& prm, int decay, unsigned grid, cudaStre
     auto k = decay == 1 ? ssd_segment_state_kernel<1, kHP>
              : decay == 2 ? ssd_segment_state_kernel<2, kHP>
                           : ssd_segment_state_kernel<0, kHP>;
-    SSD_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SPass<kHP>::kSmem));
+    if (const int st = smem_limit_once((const void*)k, (int)SPass<kHP>::kSmem)) return st;
     {
         LaunchScope ls("ssd_segment_state", s);
         k<<<grid, kSThreads, SPass<kHP>::kSmem, s>>>(prm);
@@ -1305,7 +1305,7 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
         }
         SSD_CUDA_TRY(cudaGetLastError());
     }
-    SSD_CUDA_TRY(cudaFuncSetAttribute(fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes));
+    if ((st = smem_limit_once((const void*)fused, (int)kSmemBytes)) != SSD_OK) return st;
     {
         LaunchScope ls("ssd_prefill_fused", s);
         fused<<<(unsigned)(prm.n_full + (size_t)n_split * prm.nseg), kThreads, kSmemBytes, s>>>(prm);
