@@ -297,6 +297,17 @@ SSD_API int ssd_decode_plan_launch(ssd_decode_plan* plan, void* stream);
 
 SSD_API int ssd_decode_plan_destroy(ssd_decode_plan* plan);
 
+/* n_steps decode steps as one graph launch on `stream`, with no host synchronisation inside:
+ * a plan as above is built, launched once and destroyed (the graph is freed by the driver
+ * when the launch completes).  Same arguments, layouts and errors as ssd_decode_plan_create
+ * plus the stream; every pointer, the workspace included, must stay valid until the
+ * launch has completed.  For repeated loops over the same buffers, keep a plan instead:
+ * building the graph costs host time per call. */
+SSD_API int ssd_decode_loop(int layers, int b, int H, int P, int N, int G, int kconv, int act, int io_dtype,
+                            float* h, float* conv_state, const void* xbc_ring, const float* dt_ring, int ring,
+                            const float* A, const float* D, const float* conv_w, const float* conv_b,
+                            void* y_ring, int n_steps, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------------------------
  * Measurement hooks (no counterpart on the pages; used by the benchmark)
  *

@@ -528,4 +528,18 @@ int ssd_decode_plan_destroy(ssd_decode_plan* plan) {
     return destroy_decode_plan(plan);
 }
 
+int ssd_decode_loop(int layers, int b, int H, int P, int N, int G, int kconv, int act, int io_dtype, float* h,
+                    float* conv_state, const void* xbc_ring, const float* dt_ring, int ring, const float* A,
+                    const float* D, const float* conv_w, const float* conv_b, void* y_ring, int n_steps,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+    ssd_decode_plan* plan = nullptr;
+    SSD_CHECK(ssd_decode_plan_create(&plan, layers, b, H, P, N, G, kconv, act, io_dtype, h, conv_state, xbc_ring,
+                                     dt_ring, ring, A, D, conv_w, conv_b, y_ring, n_steps, workspace,
+                                     workspace_bytes));
+    const int st = ssd_decode_plan_launch(plan, stream);
+    // an executable graph destroyed while in flight is freed when it completes
+    const int st2 = destroy_decode_plan(plan);
+    return st != SSD_OK ? st : st2;
+}
+
 }  // extern "C"

@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_decode_plan_launch.restype = _i
         L.ssd_decode_plan_destroy.argtypes = [_vp]
         L.ssd_decode_plan_destroy.restype = _i
+        L.ssd_decode_loop.argtypes = [_i] * 9 + [_vp] * 4 + [_i] + [_vp] * 5 + [_i, _vp, _sz, _vp]
+        L.ssd_decode_loop.restype = _i
         L.ssd_decode_step_noalloc.argtypes = [_i] * 9 + [_vp] * 10
         L.ssd_decode_step_noalloc.restype = _i
         L.ssd_launch_count.restype = ctypes.c_uint64
@@ -388,9 +390,19 @@ class DecodePlan:
 
 def decode_loop(h, conv_state, xbc_ring, dt_ring, A, D, conv_w, conv_b, n_steps, G=1,
                 act=SSD_ACT_SILU, stream=None):
-    """Run n_steps decode steps as one graph launch (plan built, launched, released)."""
-    plan = DecodePlan(h, conv_state, xbc_ring, dt_ring, A, D, conv_w, conv_b, n_steps, G, act)
-    y = plan.launch(stream)
+    """Run n_steps decode steps as one graph launch (ssd_decode_loop: plan built, launched,
+    released, no host synchronisation inside).  Returns y_ring [ring, layers, b, H, P]; the
+    call waits for the launch before returning because its workspace is a temporary."""
+    layers, b, H, P, N, k, Dc = _decode_shapes(h, conv_state, A, D, conv_w, conv_b, G)
+    ring = xbc_ring.shape[0]
+    _need(xbc_ring, "xbc_ring", None, (ring, layers, b, Dc))
+    io = _io(xbc_ring)
+    _need(dt_ring, "dt_ring", torch.float32, (ring, layers, b, H))
+    y_ring = torch.empty((ring, layers, b, H, P), dtype=xbc_ring.dtype, device=h.device)
+    ws = torch.empty(decode_workspace_size(layers, b, G), dtype=torch.uint8, device=h.device)
+    st = lib().ssd_decode_loop(layers, b, H, P, N, G, k, act, io, _ptr(h), _ptr(conv_state), _ptr(xbc_ring),
+                               _ptr(dt_ring), ring, _ptr(A), _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(y_ring),
+                               int(n_steps), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "ssd_decode_loop")
     torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
-    plan.close()
-    return y
+    return y_ring

@@ -148,6 +148,13 @@ def test_decode_plan_rejects():
                                     f[4], f[5], f[6], f[7], f[8], 8, f[9], 1 << 20) == INVALID
     assert L.ssd_decode_plan_launch(None, None) == INVALID
     assert L.ssd_decode_plan_destroy(None) == OK
+    # the one-call loop runs the same checks before anything is built or enqueued
+    assert L.ssd_decode_loop(1, 1, 4, 64, 128, 1, 4, 1, 1, f[0], f[1], f[2], f[3], 0, f[4], f[5], f[6], f[7],
+                             f[8], 8, f[9], 1 << 20, None) == INVALID          # ring = 0
+    assert L.ssd_decode_loop(1, 1, 4, 64, 128, 1, 4, 1, 1, f[0], f[1], f[2], f[3], 2, f[4], f[5], f[6], f[7],
+                             f[8], -1, f[9], 1 << 20, None) == INVALID         # n_steps < 0
+    assert L.ssd_decode_loop(1, 1, 4, 64, 128, 1, 4, 1, 1, f[0], f[1], f[2], f[3], 2, f[4], f[5], f[6], f[7],
+                             f[8], 8, f[9], 16, None) == WS                    # workspace too small
 
 
 def test_binding_refuses_cpu_tensors():
