@@ -1,6 +1,6 @@
 """Context-parallel prefill (tokens of every sequence split over ranks, one exchange step).
 
-CPU: two `gloo` ranks run state_space_model_04_b200.context.prefill_context_parallel -- the
+CPU: two and four `gloo` ranks run state_space_model_04_b200.context.prefill_context_parallel -- the
 same orchestration the GPUs run over NCCL -- with the steps (local state, fold, prefill)
 done by the fp64 oracle, so the exchange itself (what is gathered, in which order, which
 earlier ranks each rank folds) is checked against one whole-sequence oracle run.
@@ -13,12 +13,14 @@ import socket
 import sys
 
 import numpy as np
+import pytest
 import torch
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-SPLIT = [0, 250, 600]  # rank r holds tokens [SPLIT[r], SPLIT[r + 1])
+# rank r holds tokens [split[r], split[r + 1]): uneven shards, none a multiple of the chunk
+SPLITS = {2: [0, 250, 600], 4: [0, 100, 250, 430, 600]}
 
 
 def _free_port():
@@ -52,7 +54,7 @@ class _OracleOps:
         return torch.from_numpy(y), torch.from_numpy(h)
 
 
-def _worker(rank, world, port, out_dir):
+def _worker(rank, world, port, out_dir, split):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -60,8 +62,8 @@ def _worker(rank, world, port, out_dir):
     from ssd_inputs import make_prefill
     from state_space_model_04_b200.context import prefill_context_parallel
     dist.init_process_group("gloo", timeout=timedelta(seconds=60))
-    c = make_prefill(2, SPLIT[-1], 4, 64, 16, 2, 64, "f32", h0_std=0.1, seed=77)
-    lo, hi = SPLIT[rank], SPLIT[rank + 1]
+    c = make_prefill(2, split[-1], 4, 64, 16, 2, 64, "f32", h0_std=0.1, seed=77)
+    lo, hi = split[rank], split[rank + 1]
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float64))
     y, h = prefill_context_parallel(t(c.x[:, lo:hi]), t(c.dt[:, lo:hi]), t(c.A), t(c.B[:, lo:hi]),
                                     t(c.C[:, lo:hi]), t(c.D), h0=t(c.h0), ops=_OracleOps)
@@ -70,20 +72,23 @@ def _worker(rank, world, port, out_dir):
     np.save(os.path.join(out_dir, "h%d.npy" % rank), h.numpy())
 
 
-def test_two_gloo_ranks_context_parallel_prefill(tmp_path):
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_context_parallel_prefill(world, tmp_path):
     import oracle
     from ssd_inputs import make_prefill
-    world, port = 2, _free_port()
-    mp.start_processes(_worker, args=(world, port, str(tmp_path)), nprocs=world, join=True, start_method="spawn")
-    c = make_prefill(2, SPLIT[-1], 4, 64, 16, 2, 64, "f32", h0_std=0.1, seed=77)
+    split, port = SPLITS[world], _free_port()
+    mp.start_processes(_worker, args=(world, port, str(tmp_path), split), nprocs=world, join=True,
+                       start_method="spawn")
+    c = make_prefill(2, split[-1], 4, 64, 16, 2, 64, "f32", h0_std=0.1, seed=77)
     y_ref, h_ref = oracle.ssd_recurrence(c.x, c.dt, c.A, c.B, c.C, c.D, c.h0)
     y = np.concatenate([np.load(tmp_path / ("y%d.npy" % r)) for r in range(world)], axis=1)
     np.testing.assert_allclose(y, y_ref, rtol=1e-9, atol=1e-9 * np.abs(y_ref).max())
-    np.testing.assert_allclose(np.load(tmp_path / "h1.npy"), h_ref, rtol=1e-9, atol=1e-12)
-    # rank 0's state is the state after its own tokens, not the sequence's
-    _, h_first = oracle.ssd_recurrence(c.x[:, :SPLIT[1]], c.dt[:, :SPLIT[1]], c.A, c.B[:, :SPLIT[1]],
-                                       c.C[:, :SPLIT[1]], c.D, c.h0)
-    np.testing.assert_allclose(np.load(tmp_path / "h0.npy"), h_first, rtol=1e-9, atol=1e-12)
+    # every rank's state is the state after its own last token, not the sequence's
+    for r in range(world):
+        hi = split[r + 1]
+        _, h_r = oracle.ssd_recurrence(c.x[:, :hi], c.dt[:, :hi], c.A, c.B[:, :hi], c.C[:, :hi], c.D, c.h0)
+        np.testing.assert_allclose(np.load(tmp_path / ("h%d.npy" % r)), h_r, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(np.load(tmp_path / ("h%d.npy" % (world - 1))), h_ref, rtol=1e-9, atol=1e-12)
 
 
 def test_single_process_is_a_plain_prefill():
