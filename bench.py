@@ -39,6 +39,8 @@ sys.path.insert(0, ROOT)
 METRIC = "SSD prefill TFLOP/s + tokens/s; decode steps/s + HBM GB/s; % of roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal B200 figures, for context beside the measured ones: HBM3e per the HGX spec sheet
+NOMINAL_HBM_GBS = 7700.0
 
 # prefill workload (the 2.7B-layer configuration)
 PB, PT, PH, PP, PN, PG, PL = 8, 4096, 80, 64, 128, 1, 256
@@ -398,6 +400,9 @@ def main():
                 "tensor_tflops": flops / (dom_avg_ms * 1e-3) / 1e12 if dom_name == "ssd_prefill_fused" else None,
                 "tensor_frac_of_bf16_peak": (flops / (dom_avg_ms * 1e-3) / 1e12 / pk["bf16_tflops"])
                 if dom_name == "ssd_prefill_fused" else None,
+                "tensor_frac_of_bf16_sustained": (flops / (dom_avg_ms * 1e-3) / 1e12 / pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+                if dom_name == "ssd_prefill_fused" else None,
+                "frac_of_nominal_hbm": achieved / NOMINAL_HBM_GBS, "nominal_hbm_gbs": NOMINAL_HBM_GBS,
                 "kernels": {k: {"launches": v[0], "avg_ms": v[1] / max(v[0], 1)} for k, v in kt.items()}}
 
     # ---------------- the same step from the raw time step (dt pre-processing fused into the
@@ -681,6 +686,7 @@ def bench_decode(ssd, torch, dev, stream, case, hf, b, args, clocks, barrier, ma
     return {"batch": b, "layers": DL, "steps": steps, "steps_per_launch": steps_per_launch,
             "steps_per_s": sps, "tokens_per_s": sps * b, "ms_per_step": ms / steps,
             "bytes_per_step": byt, "hbm_gbs_alg": gbs, "hbm_frac": gbs / world / pk["hbm_gbs"],
+            "hbm_frac_of_nominal": gbs / world / NOMINAL_HBM_GBS,
             "kernel": "decode_step (graph of %d steps)" % steps_per_launch, "state_finite": ok,
             "loop_compare": loops}
 
