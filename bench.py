@@ -367,8 +367,11 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     w0 = time.time()
     e0.record(stream)
+    step_ev = []  # an event after every step: per-step times (best and median) ride along
     for _ in range(args.steps):
         prefill_step()
+        step_ev.append(torch.cuda.Event(enable_timing=True))
+        step_ev[-1].record(stream)
     e1.record(stream)
     torch.cuda.synchronize()
     clocks.mark(w0, time.time())
@@ -376,6 +379,9 @@ def main():
     launches = ssd.launch_count() - n0
     barrier()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    step_ms = sorted((e0 if i == 0 else step_ev[i - 1]).elapsed_time(step_ev[i]) for i in range(args.steps))
+    step_stats = {"best": max_over_ranks(step_ms[0]), "median": max_over_ranks(step_ms[len(step_ms) // 2]),
+                  "steps": args.steps}
     # dominant kernel: the one with the largest summed event time in the timed region
     dom = max(kt.items(), key=lambda kv: kv[1][1])
     dom_name, (dom_n, dom_ms) = dom
@@ -527,7 +533,7 @@ def main():
                            "G": PG, "chunk": PL, "global_batch": PB * world, "seq_len": PT,
                            "parallelism": "dp%d" % world,
                            "l2": "inputs larger than L2 (%.0f MB per step vs 126 MB)" % (pbytes / 1e6)},
-                "tokens_per_s": tokens_s, "flops_per_step": flops, "chunk_executed": exec_L,
+                "tokens_per_s": tokens_s, "step_ms": step_stats, "flops_per_step": flops, "chunk_executed": exec_L,
                 "tflops_at_requested_chunk": job_rate(flops_req, world, ms) / 1e12, "bytes_per_step": pbytes,
                 "hbm_gbs_alg": pbytes * world / (ms * 1e-3) / 1e9,
                 "tensor_frac": tflops / world / pk["bf16_tflops"],
