@@ -284,34 +284,63 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
         "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(bar)
         : "memory");
 }
-#define SSD_TMEM_LD32(taddr, r)                                                                          \
-    asm volatile(                                                                                        \
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15," \
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                      \
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),           \
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),        \
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),     \
-          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),     \
-          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                              \
-        : "r"(taddr))
-#define SSD_TMEM_LD16(taddr, r)                                                                          \
-    asm volatile(                                                                                        \
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}," \
-        " [%16];"                                                                                        \
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),           \
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),        \
-          "=r"(r[14]), "=r"(r[15])                                                                        \
-        : "r"(taddr))
-#define SSD_TMEM_ST16(taddr, r)                                                                          \
-    asm volatile(                                                                                        \
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"  \
-        "%15,%16};"                                                                                      \
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),      \
-          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),   \
-          "r"(r[15])                                                                                      \
+// TMEM <-> register moves.  tcgen05.ld writes its destination registers, and tcgen05.st
+// reads its source registers, asynchronously until the matching tcgen05.wait; each macro
+// issues the moves and the wait in ONE asm statement, so the compiler never sees the
+// registers as defined (or free) before the wait and cannot reuse, spill or read them
+// while the move is still in flight.
+#define SSD_TMEM_LD32_WAIT(taddr, r) \
+    asm volatile( \
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t" \
+        "tcgen05.wait::ld.sync.aligned;" \
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), \
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), \
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), \
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), \
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31]) \
+        : "r"(taddr) \
         : "memory")
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+#define SSD_TMEM_LD32x2_WAIT(ta, ra, tb, rb) \
+    asm volatile( \
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t" \
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t" \
+        "tcgen05.wait::ld.sync.aligned;" \
+        : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]), "=r"(ra[6]), \
+          "=r"(ra[7]), "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]), "=r"(ra[12]), "=r"(ra[13]), \
+          "=r"(ra[14]), "=r"(ra[15]), "=r"(ra[16]), "=r"(ra[17]), "=r"(ra[18]), "=r"(ra[19]), "=r"(ra[20]), \
+          "=r"(ra[21]), "=r"(ra[22]), "=r"(ra[23]), "=r"(ra[24]), "=r"(ra[25]), "=r"(ra[26]), "=r"(ra[27]), \
+          "=r"(ra[28]), "=r"(ra[29]), "=r"(ra[30]), "=r"(ra[31]), "=r"(rb[0]), "=r"(rb[1]), "=r"(rb[2]), \
+          "=r"(rb[3]), "=r"(rb[4]), "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]), "=r"(rb[8]), "=r"(rb[9]), \
+          "=r"(rb[10]), "=r"(rb[11]), "=r"(rb[12]), "=r"(rb[13]), "=r"(rb[14]), "=r"(rb[15]), "=r"(rb[16]), \
+          "=r"(rb[17]), "=r"(rb[18]), "=r"(rb[19]), "=r"(rb[20]), "=r"(rb[21]), "=r"(rb[22]), "=r"(rb[23]), \
+          "=r"(rb[24]), "=r"(rb[25]), "=r"(rb[26]), "=r"(rb[27]), "=r"(rb[28]), "=r"(rb[29]), "=r"(rb[30]), \
+          "=r"(rb[31]) \
+        : "r"(ta), "r"(tb) \
+        : "memory")
+#define SSD_TMEM_LD16x2_WAIT(ta, ra, tb, rb) \
+    asm volatile( \
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t" \
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t" \
+        "tcgen05.wait::ld.sync.aligned;" \
+        : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]), "=r"(ra[6]), \
+          "=r"(ra[7]), "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]), "=r"(ra[12]), "=r"(ra[13]), \
+          "=r"(ra[14]), "=r"(ra[15]), "=r"(rb[0]), "=r"(rb[1]), "=r"(rb[2]), "=r"(rb[3]), "=r"(rb[4]), \
+          "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]), "=r"(rb[8]), "=r"(rb[9]), "=r"(rb[10]), "=r"(rb[11]), \
+          "=r"(rb[12]), "=r"(rb[13]), "=r"(rb[14]), "=r"(rb[15]) \
+        : "r"(ta), "r"(tb) \
+        : "memory")
+#define SSD_TMEM_ST16x2_WAIT(ta, ra, tb, rb) \
+    asm volatile( \
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17};\n\t" \
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%1], {%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};\n\t" \
+        "tcgen05.wait::st.sync.aligned;" \
+        : \
+        : "r"(ta), "r"(tb), "r"(ra[0]), "r"(ra[1]), "r"(ra[2]), "r"(ra[3]), "r"(ra[4]), "r"(ra[5]), \
+          "r"(ra[6]), "r"(ra[7]), "r"(ra[8]), "r"(ra[9]), "r"(ra[10]), "r"(ra[11]), "r"(ra[12]), \
+          "r"(ra[13]), "r"(ra[14]), "r"(ra[15]), "r"(rb[0]), "r"(rb[1]), "r"(rb[2]), "r"(rb[3]), \
+          "r"(rb[4]), "r"(rb[5]), "r"(rb[6]), "r"(rb[7]), "r"(rb[8]), "r"(rb[9]), "r"(rb[10]), "r"(rb[11]), \
+          "r"(rb[12]), "r"(rb[13]), "r"(rb[14]), "r"(rb[15]) \
+        : "memory")
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -544,9 +573,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t ry[16], rs[16];
-                SSD_TMEM_LD16(tmem + lane_addr + kColY + (k & 1) * 64 + p0 + hh * 16, ry);
-                SSD_TMEM_LD16(tmem + lane_addr + kColYst + (k & 1) * 64 + p0 + hh * 16, rs);
-                tmem_wait_ld();
+                SSD_TMEM_LD16x2_WAIT(tmem + lane_addr + kColY + (k & 1) * 64 + p0 + hh * 16, ry,
+                                     tmem + lane_addr + kColYst + (k & 1) * 64 + p0 + hh * 16, rs);
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     yp[hh * 8 + j] = pack_bf16(fmaf(ei, __uint_as_float(rs[2 * j]), __uint_as_float(ry[2 * j])),
@@ -591,8 +619,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                     const int c = (half == q) ? half + 2 * (1 - cc) : half + 2 * cc;
                     uint32_t raw[32];
                     if (c <= q) {
-                        SSD_TMEM_LD32(tmem + lane_addr + kColCB + c * 32, raw);
-                        tmem_wait_ld();
+                        SSD_TMEM_LD32_WAIT(tmem + lane_addr + kColCB + c * 32, raw);
                     }
                     if (cc == 1) {
                         tc_fence_before();
@@ -632,9 +659,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 if (live) {
                     tc_fence_after();
                     const int cfirst = (half == q) ? half + 2 : half;
-                    SSD_TMEM_ST16(tmem + lane_addr + kColP + cfirst * 16, pk[0]);
-                    SSD_TMEM_ST16(tmem + lane_addr + kColP + (2 * half + 2 - cfirst) * 16, pk[1]);
-                    tmem_wait_st();
+                    SSD_TMEM_ST16x2_WAIT(tmem + lane_addr + kColP + cfirst * 16, pk[0],
+                                         tmem + lane_addr + kColP + (2 * half + 2 - cfirst) * 16, pk[1]);
                     tc_fence_before();
                     mbar_arrive(bar(BAR_SCORES));
                 }
@@ -720,8 +746,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 tc_fence_after();
                 {
                     uint32_t raw[32];
-                    SSD_TMEM_LD32(tmem + lane_addr + kColS + p0, raw);
-                    tmem_wait_ld();
+                    SSD_TMEM_LD32_WAIT(tmem + lane_addr + kColS + p0, raw);
                     const float gam = dexp<kDecay>(__expf(cs_last_prev));
 #pragma unroll
                     for (int j = 0; j < 32; ++j) Hs[j] = fmaf(gam, Hs[j], __uint_as_float(raw[j]));
@@ -989,12 +1014,12 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
             constexpr int kCols = 32 * kHP;  // 32 (half of one head) or 64 (a whole head)
             const int pbase = kHP == 2 ? 0 : half * 32;
             uint32_t raw[kCols];
-            SSD_TMEM_LD32(tmem + lane_addr + h * 64 + pbase, raw);
             if constexpr (kHP == 2) {
                 uint32_t* raw_hi = raw + 32;
-                SSD_TMEM_LD32(tmem + lane_addr + h * 64 + 32, raw_hi);
+                SSD_TMEM_LD32x2_WAIT(tmem + lane_addr + h * 64, raw, tmem + lane_addr + h * 64 + 32, raw_hi);
+            } else {
+                SSD_TMEM_LD32_WAIT(tmem + lane_addr + h * 64 + pbase, raw);
             }
-            tmem_wait_ld();
             tc_fence_before();
             if (!*s_abort) {
                 const size_t o = (size_t)(su0 + h) * (prm.nseg - 1) + seg;
