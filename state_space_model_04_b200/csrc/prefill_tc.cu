@@ -378,7 +378,9 @@ __device__ __forceinline__ float block_cumsum(float a, int q, int lane, bool pub
 }
 
 // ------------------------------------------------------------------ kernel
-template <int kDecay>
+// kRawDt: dt arrives raw (the DtMap pre-processing applies); it is then formed where a block
+// uses it rather than where it is prefetched, so the prefetch still hides the load.
+template <int kDecay, bool kRawDt = false>
 __global__ void __launch_bounds__(kThreads, 1)
 ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -707,7 +709,11 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         bool stopped = false;
         auto load_dt = [&](int u) {
             const int tok = tb + u * kBlk + r;
-            return (u < nblk && tok < T) ? dt_value(__ldg(prm.dt + ((size_t)bi * T + tok) * H + hd), prm.dtm, hd) : 0.f;
+            if constexpr (kRawDt)
+                return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;
+            else
+                return (u < nblk && tok < T) ? dt_value(__ldg(prm.dt + ((size_t)bi * T + tok) * H + hd), prm.dtm, hd)
+                                             : 0.f;
         };
         // dt is fetched two blocks ahead: under full HBM load its latency is microseconds
         float dt_a = load_dt(0), dt_b = load_dt(1);
@@ -715,7 +721,11 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         // iteration k: inputs of block k+1 (w o X), state and output of block k
         for (int k = -1; k < nblk; ++k) {
             const int s = (k + 1) & 1;
-            const float dtv = dt_a;
+            float dtv = dt_a;
+            if constexpr (kRawDt) {  // raw dt of block k+1, formed now (0 past the end)
+                const int tok = tb + (k + 1) * kBlk + r;
+                dtv = (k + 1 < nblk && tok < T) ? dt_value(dt_a, prm.dtm, hd) : 0.f;
+            }
             dt_a = dt_b;
             dt_b = load_dt(k + 3);
             if (!live || *s_abort) s_ystop[s] = 1;
@@ -1296,8 +1306,12 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     prm.dt = dt;
     prm.dtm = dtm;
     const int decay = g_decay_mode.load();
-    auto fused = decay == 1 ? ssd_prefill_fused_kernel<1> : decay == 2 ? ssd_prefill_fused_kernel<2>
-                                                                        : ssd_prefill_fused_kernel<0>;
+    auto fused = dtm.raw ? (decay == 1   ? ssd_prefill_fused_kernel<1, true>
+                            : decay == 2 ? ssd_prefill_fused_kernel<2, true>
+                                         : ssd_prefill_fused_kernel<0, true>)
+                         : (decay == 1   ? ssd_prefill_fused_kernel<1, false>
+                            : decay == 2 ? ssd_prefill_fused_kernel<2, false>
+                                         : ssd_prefill_fused_kernel<0, false>);
     prm.A = A;
     prm.D = D;
     prm.h0 = h0;
