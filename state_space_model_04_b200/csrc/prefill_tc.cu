@@ -973,9 +973,11 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
         constexpr int kChunks = 8 / (3 - kHP);  // 16-byte chunks of an X row per thread: 4 or 8
         const int c0 = kHP == 2 ? 0 : half * 4;
         const float Ah = prm.A[hd];
+        // dt as stored (raw when the DtMap pre-processing applies), fetched two blocks ahead and
+        // formed where the block uses it, so the prefetch is never waited on early
         auto load_dt = [&](int u) {
             const int tok = block_t0(u) + r;
-            return (u < nblk && tok < T) ? dt_value(__ldg(prm.dt + ((size_t)bi * T + tok) * H + hd), prm.dtm, hd) : 0.f;
+            return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;
         };
         bool live = __all_sync(0xffffffffu, !*s_abort);
         bool stopped = false;
@@ -983,7 +985,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
         float later = 0.f;  // log decay from the end of the current block to the end of the segment
         for (int u = 0; u < nblk; ++u) {
             const int s = u & 1;  // stop-flag and quadrant-sum buffer
-            const float dtv = dt_a;
+            const float dtv = block_t0(u) + r < T ? dt_value(dt_a, prm.dtm, hd) : 0.f;
             dt_a = dt_b;
             dt_b = load_dt(u + 2);
             if (!live || *s_abort) s_ystop[s] = 1;
