@@ -712,11 +712,10 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             if constexpr (kRawDt)
                 return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;
             else
-                return (u < nblk && tok < T) ? dt_value(__ldg(prm.dt + ((size_t)bi * T + tok) * H + hd), prm.dtm, hd)
-                                             : 0.f;
+                return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;  // used as given
         };
-        // dt is fetched two blocks ahead: under full HBM load its latency is microseconds
-        float dt_a = load_dt(0), dt_b = load_dt(1);
+        // dt is fetched three blocks ahead: under full HBM load its latency is microseconds
+        float dt_a = load_dt(0), dt_b = load_dt(1), dt_c = load_dt(2);
         float cs_last_prev = 0.f;  // total of the block whose state update is next
         // iteration k: inputs of block k+1 (w o X), state and output of block k
         for (int k = -1; k < nblk; ++k) {
@@ -727,7 +726,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 dtv = (k + 1 < nblk && tok < T) ? dt_value(dt_a, prm.dtm, hd) : 0.f;
             }
             dt_a = dt_b;
-            dt_b = load_dt(k + 3);
+            dt_b = dt_c;
+            dt_c = load_dt(k + 4);
             if (!live || *s_abort) s_ystop[s] = 1;
             float cend[4], cs_last;
             float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_ytot + s * 4, 3, cs_last, cend);
