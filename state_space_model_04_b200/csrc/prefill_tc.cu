@@ -226,6 +226,35 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// TMEM allocation for the whole CTA; returns the allocation's address (the same in every
+// thread).  tcgen05.alloc writes the address into a shared-memory slot.  The slot first
+// holds a sentinel, ordered before the allocation by a barrier, and every thread re-reads
+// it until the address has replaced the sentinel (bounded).  So no thread acts on a value
+// that predates the allocation -- what a CTA's first read may otherwise return is whatever
+// that shared memory held before, benign after an earlier CTA of the same kernel and
+// garbage on a GPU's first launch.  An address that never arrives leaves the sentinel,
+// which the caller treats as a failed CTA (status SSD_ERR_INTERNAL).
+constexpr uint32_t kTmemSentinel = 0xFFFFFFFFu;
+__device__ __forceinline__ uint32_t tmem_alloc_cta(uint32_t* s_tmem, uint32_t cols, bool alloc_warp) {
+    volatile uint32_t* slot = s_tmem;
+    if (threadIdx.x == 0) *slot = kTmemSentinel;
+    __syncthreads();
+    if (alloc_warp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
+                     "r"(cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    uint32_t t = *slot;
+    if (t == kTmemSentinel) {
+        const unsigned long long t0 = globaltimer();
+        while (t == kTmemSentinel && globaltimer() - t0 < kWaitLimitNs) t = *slot;
+    }
+    return t;
+}
 __device__ __forceinline__ void group_bar(int id) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kGroupThreads) : "memory");
 }
@@ -288,7 +317,10 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
 // reads its source registers, asynchronously until the matching tcgen05.wait; each macro
 // issues the moves and the wait in ONE asm statement, so the compiler never sees the
 // registers as defined (or free) before the wait and cannot reuse, spill or read them
-// while the move is still in flight.
+// while the move is still in flight.  The two-load forms take the second address as an
+// immediate offset from the first and form it in a register of their own before the first
+// load issues: an output of the first load, written asynchronously, can then never be the
+// register the second load reads its address from.
 #define SSD_TMEM_LD32_WAIT(taddr, r) \
     asm volatile( \
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t" \
@@ -300,11 +332,12 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31]) \
         : "r"(taddr) \
         : "memory")
-#define SSD_TMEM_LD32x2_WAIT(ta, ra, tb, rb) \
+#define SSD_TMEM_LD32x2_WAIT(ta, off, ra, rb) \
     asm volatile( \
+        "{\n\t.reg .b32 tb;\n\tadd.u32 tb, %64, %65;\n\t" \
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t" \
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t" \
-        "tcgen05.wait::ld.sync.aligned;" \
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [tb];\n\t" \
+        "tcgen05.wait::ld.sync.aligned;\n\t}" \
         : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]), "=r"(ra[6]), \
           "=r"(ra[7]), "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]), "=r"(ra[12]), "=r"(ra[13]), \
           "=r"(ra[14]), "=r"(ra[15]), "=r"(ra[16]), "=r"(ra[17]), "=r"(ra[18]), "=r"(ra[19]), "=r"(ra[20]), \
@@ -315,19 +348,20 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
           "=r"(rb[17]), "=r"(rb[18]), "=r"(rb[19]), "=r"(rb[20]), "=r"(rb[21]), "=r"(rb[22]), "=r"(rb[23]), \
           "=r"(rb[24]), "=r"(rb[25]), "=r"(rb[26]), "=r"(rb[27]), "=r"(rb[28]), "=r"(rb[29]), "=r"(rb[30]), \
           "=r"(rb[31]) \
-        : "r"(ta), "r"(tb) \
+        : "r"(ta), "n"(off) \
         : "memory")
-#define SSD_TMEM_LD16x2_WAIT(ta, ra, tb, rb) \
+#define SSD_TMEM_LD16x2_WAIT(ta, off, ra, rb) \
     asm volatile( \
+        "{\n\t.reg .b32 tb;\n\tadd.u32 tb, %32, %33;\n\t" \
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t" \
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t" \
-        "tcgen05.wait::ld.sync.aligned;" \
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [tb];\n\t" \
+        "tcgen05.wait::ld.sync.aligned;\n\t}" \
         : "=r"(ra[0]), "=r"(ra[1]), "=r"(ra[2]), "=r"(ra[3]), "=r"(ra[4]), "=r"(ra[5]), "=r"(ra[6]), \
           "=r"(ra[7]), "=r"(ra[8]), "=r"(ra[9]), "=r"(ra[10]), "=r"(ra[11]), "=r"(ra[12]), "=r"(ra[13]), \
           "=r"(ra[14]), "=r"(ra[15]), "=r"(rb[0]), "=r"(rb[1]), "=r"(rb[2]), "=r"(rb[3]), "=r"(rb[4]), \
           "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]), "=r"(rb[8]), "=r"(rb[9]), "=r"(rb[10]), "=r"(rb[11]), \
           "=r"(rb[12]), "=r"(rb[13]), "=r"(rb[14]), "=r"(rb[15]) \
-        : "r"(ta), "r"(tb) \
+        : "r"(ta), "n"(off) \
         : "memory")
 #define SSD_TMEM_ST16x2_WAIT(ta, ra, tb, rb) \
     asm volatile( \
@@ -429,15 +463,11 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         s_ystop[0] = s_ystop[1] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) {  // TMEM allocation (whole warp)
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
-                     "r"(kTmemCols));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    const uint32_t tmem = tmem_alloc_cta(s_tmem, kTmemCols, warp == 1);  // warp 1 owns the TMEM
+    if (tmem == kTmemSentinel) {
+        *s_abort = 1;
+        atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (3 << 8));
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *s_tmem;
 
     if (warp == 0) {
         // ================================================================ TMA producer
@@ -575,8 +605,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t ry[16], rs[16];
-                SSD_TMEM_LD16x2_WAIT(tmem + lane_addr + kColY + (k & 1) * 64 + p0 + hh * 16, ry,
-                                     tmem + lane_addr + kColYst + (k & 1) * 64 + p0 + hh * 16, rs);
+                SSD_TMEM_LD16x2_WAIT(tmem + lane_addr + kColY + (k & 1) * 64 + p0 + hh * 16, kColYst - kColY, ry, rs);
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     yp[hh * 8 + j] = pack_bf16(fmaf(ei, __uint_as_float(rs[2 * j]), __uint_as_float(ry[2 * j])),
@@ -714,8 +743,9 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             else
                 return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;  // used as given
         };
-        // dt is fetched three blocks ahead: under full HBM load its latency is microseconds
-        float dt_a = load_dt(0), dt_b = load_dt(1), dt_c = load_dt(2);
+        // dt is fetched four blocks ahead: it is a strided gather, and under full HBM load its
+        // latency is microseconds
+        float dt_a = load_dt(0), dt_b = load_dt(1), dt_c = load_dt(2), dt_d = load_dt(3);
         float cs_last_prev = 0.f;  // total of the block whose state update is next
         // iteration k: inputs of block k+1 (w o X), state and output of block k
         for (int k = -1; k < nblk; ++k) {
@@ -727,7 +757,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
             }
             dt_a = dt_b;
             dt_b = dt_c;
-            dt_c = load_dt(k + 4);
+            dt_c = dt_d;
+            dt_d = load_dt(k + 5);
             if (!live || *s_abort) s_ystop[s] = 1;
             float cend[4], cs_last;
             float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_ytot + s * 4, 3, cs_last, cend);
@@ -825,7 +856,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     // then is the TMEM released.
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 1 && tmem != kTmemSentinel) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
@@ -906,15 +937,11 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
         s_ystop[0] = s_ystop[1] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
-                     "r"(SP::kTmemCols));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    const uint32_t tmem = tmem_alloc_cta(s_tmem, SP::kTmemCols, warp == 1);  // warp 1 owns the TMEM
+    if (tmem == kTmemSentinel) {
+        *s_abort = 1;
+        atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (4 << 8));
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *s_tmem;
     constexpr int kS = SP::kSlots;
 
     if (warp == 0) {
@@ -1028,7 +1055,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
             uint32_t raw[kCols];
             if constexpr (kHP == 2) {
                 uint32_t* raw_hi = raw + 32;
-                SSD_TMEM_LD32x2_WAIT(tmem + lane_addr + h * 64, raw, tmem + lane_addr + h * 64 + 32, raw_hi);
+                SSD_TMEM_LD32x2_WAIT(tmem + lane_addr + h * 64, 32, raw, raw_hi);
             } else {
                 SSD_TMEM_LD32_WAIT(tmem + lane_addr + h * 64 + pbase, raw);
             }
@@ -1045,7 +1072,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 1 && tmem != kTmemSentinel) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(SP::kTmemCols));
     }
