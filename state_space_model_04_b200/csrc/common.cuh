@@ -40,11 +40,14 @@ struct DtMap {
     float lo, hi;       // clamp range (hi may be +inf)
     int raw;            // 0: dt is used as given
 };
-__device__ __forceinline__ float dt_value(float v, const DtMap& m, int h) {
-    if (!m.raw) return v;
-    const float z = v + (m.bias ? __ldg(m.bias + h) : 0.f);
+// clamp(softplus(z)) for z = dt_raw + the head's bias
+__device__ __forceinline__ float dt_softplus_clamp(float z, const DtMap& m) {
     const float sp = z > 20.f ? z : log1pf(expf(z));
     return fminf(fmaxf(sp, m.lo), m.hi);
+}
+__device__ __forceinline__ float dt_value(float v, const DtMap& m, int h) {
+    if (!m.raw) return v;
+    return dt_softplus_clamp(v + (m.bias ? __ldg(m.bias + h) : 0.f), m);
 }
 
 // Map a CUDA error to a status with detail.

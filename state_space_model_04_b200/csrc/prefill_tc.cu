@@ -746,15 +746,19 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         // dt is fetched four blocks ahead: it is a strided gather, and under full HBM load its
         // latency is microseconds
         float dt_a = load_dt(0), dt_b = load_dt(1), dt_c = load_dt(2), dt_d = load_dt(3);
+        // raw dt: the head's bias is loaded once, and each block's dt is formed one iteration
+        // before the block needs it, ahead of that iteration's waits (0 past the end)
+        const float dt_bias = (kRawDt && prm.dtm.bias) ? __ldg(prm.dtm.bias + hd) : 0.f;
+        auto form_dt = [&](int u, float v) {
+            const int tok = tb + u * kBlk + r;
+            return (u < nblk && tok < T) ? dt_softplus_clamp(v + dt_bias, prm.dtm) : 0.f;
+        };
+        float dt_next = kRawDt ? form_dt(0, dt_a) : 0.f;
         float cs_last_prev = 0.f;  // total of the block whose state update is next
         // iteration k: inputs of block k+1 (w o X), state and output of block k
         for (int k = -1; k < nblk; ++k) {
             const int s = (k + 1) & 1;
-            float dtv = dt_a;
-            if constexpr (kRawDt) {  // raw dt of block k+1, formed now (0 past the end)
-                const int tok = tb + (k + 1) * kBlk + r;
-                dtv = (k + 1 < nblk && tok < T) ? dt_value(dt_a, prm.dtm, hd) : 0.f;
-            }
+            const float dtv = kRawDt ? dt_next : dt_a;  // dt of block k+1
             dt_a = dt_b;
             dt_b = dt_c;
             dt_c = dt_d;
@@ -768,6 +772,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) cend[c] = dlog<kDecay>(cend[c]);
             }
+            if constexpr (kRawDt) dt_next = form_dt(k + 2, dt_a);  // dt_a now holds block k+2's
             if (s_ystop[s]) { stopped = true; break; }
             // ---- w o X of block k+1 (needs S^T(k) accumulated: the MMA has read Xs(k))
             if (live && k >= 0) live = warp_wait(bar(BAR_ACCS), k & 1, s_abort, prm.status, 13);
@@ -1009,10 +1014,12 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
         bool live = __all_sync(0xffffffffu, !*s_abort);
         bool stopped = false;
         float dt_a = load_dt(0), dt_b = load_dt(1);
+        const float dt_bias = (prm.dtm.raw && prm.dtm.bias) ? __ldg(prm.dtm.bias + hd) : 0.f;  // loaded once
         float later = 0.f;  // log decay from the end of the current block to the end of the segment
         for (int u = 0; u < nblk; ++u) {
             const int s = u & 1;  // stop-flag and quadrant-sum buffer
-            const float dtv = block_t0(u) + r < T ? dt_value(dt_a, prm.dtm, hd) : 0.f;
+            const float dtv =
+                block_t0(u) + r < T ? (prm.dtm.raw ? dt_softplus_clamp(dt_a + dt_bias, prm.dtm) : dt_a) : 0.f;
             dt_a = dt_b;
             dt_b = load_dt(u + 2);
             if (!live || *s_abort) s_ystop[s] = 1;
