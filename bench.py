@@ -437,8 +437,9 @@ def main():
     barrier()
     ms_raw = max_over_ranks(e0r.elapsed_time(e1r) / n_raw)
     dt_raw_entry = {"ms_per_step": ms_raw, "vs_preprocessed_dt": ms_raw / ms,
-                    "note": "softplus(dt_raw + dt_bias) formed inside the kernels (raw dt prefetched, formed "
-                            "where a block uses it); no separate pass"}
+                    "note": "softplus(dt_raw + dt_bias) formed inside the kernels (raw dt prefetched; the fused "
+                            "kernel forms each block's dt one iteration before the block uses it); "
+                            "no separate pass"}
     del dt_raw
     prefill_step()  # leave y / h_final as the headline step computes them
     torch.cuda.synchronize()

@@ -169,7 +169,9 @@ SSD_API int ssd_prefill_context_scan(int world, int rank, int b, int H, int P, i
 /* Synchronises `stream` and returns the device-side status recorded by the most recent
  * ssd_prefill that used `workspace` (SSD_OK, or SSD_ERR_TIMEOUT if a bounded wait inside
  * the tensor-core kernel expired, or SSD_ERR_INTERNAL for a failed device consistency
- * check), then clears it.  Each ssd_prefill call resets the status word first. */
+ * check: a dynamic shared-memory base that is not 1024-byte aligned, or a tensor-memory
+ * allocation whose address never reached the CTA), then clears it; ssd_last_error names
+ * the wait site or the check.  Each ssd_prefill call resets the status word first. */
 SSD_API int ssd_prefill_check(void* workspace, void* stream);
 
 /* Failure-detection test hook.  Arms a one-shot fault for the next ssd_prefill in this

@@ -227,12 +227,12 @@ __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 // TMEM allocation for the whole CTA; returns the allocation's address (the same in every
-// thread).  tcgen05.alloc writes the address into a shared-memory slot.  The slot first
-// holds a sentinel, ordered before the allocation by a barrier, and every thread re-reads
-// it until the address has replaced the sentinel (bounded).  So no thread acts on a value
-// that predates the allocation -- what a CTA's first read may otherwise return is whatever
-// that shared memory held before, benign after an earlier CTA of the same kernel and
-// garbage on a GPU's first launch.  An address that never arrives leaves the sentinel,
+// thread).  tcgen05.alloc writes the address into a shared-memory slot, which the fence /
+// barrier / fence sequence orders before the read.  As a guard on top of that, the slot
+// first holds a sentinel (written before the allocation, ordered by a barrier) and every
+// thread re-reads it until the address has replaced it (bounded), so no thread can act on
+// whatever that shared memory held before the allocation; a diagnostic build that counted
+// first reads of the sentinel saw none.  An address that never arrives leaves the sentinel,
 // which the caller treats as a failed CTA (status SSD_ERR_INTERNAL).
 constexpr uint32_t kTmemSentinel = 0xFFFFFFFFu;
 __device__ __forceinline__ uint32_t tmem_alloc_cta(uint32_t* s_tmem, uint32_t cols, bool alloc_warp) {
@@ -1463,6 +1463,14 @@ int prefill_tc_status(void* ws, cudaStream_t s) {
     if (v == 0) return SSD_OK;
     SSD_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), s));
     const int code = v & 0xff, where = v >> 8;
+    if (code == SSD_ERR_INTERNAL) {
+        const char* what = where == 1   ? "fused kernel: dynamic shared memory not 1024-byte aligned"
+                           : where == 2 ? "segment state pass: dynamic shared memory not 1024-byte aligned"
+                           : where == 3 ? "fused kernel: tensor-memory address never arrived"
+                           : where == 4 ? "segment state pass: tensor-memory address never arrived"
+                                        : "unknown check";
+        return set_error(code, "device consistency check %d failed (%s)", where, what);
+    }
     return set_error(code, "device status %d at wait site %d", code, where);
 }
 
