@@ -54,6 +54,7 @@ def _load():
         lib.oracle_ssd_chunked.argtypes = [i] * 7 + [_dp] * 9 + [i]
         lib.oracle_ssd_quadratic.argtypes = [i] * 6 + [_dp] * 9 + [i]
         lib.oracle_decode_step.argtypes = [i] * 8 + [_dp] * 9 + [i]
+        lib.oracle_decode_step_mag.argtypes = [i] * 8 + [_dp] * 9 + [i]
         lib.oracle_max_threads.restype = ctypes.c_int
         lib.oracle_dt_from_raw.argtypes = [ctypes.c_size_t, i, _dp, _dp, ctypes.c_double, ctypes.c_double, _dp]
         _lib = lib
@@ -104,6 +105,42 @@ def ssd_chunked(x, dt, A, B, C, D, L, h0=None, nthreads=0):
 def ssd_quadratic(x, dt, A, B, C, D, h0=None, nthreads=0):
     """Whole-sequence quadratic form (one chunk of length T, direct segment sums)."""
     return _prefill(_load().oracle_ssd_quadratic, x, dt, A, B, C, D, h0, None, nthreads)
+
+
+def ssd_magnitudes(x, dt, A, B, C, D, h0=None, nthreads=0):
+    """Sum of the absolute values of the terms behind every output of the prefill, (y_mag,
+    h_final_mag) in float64: the scale of the rounding error an evaluation of the outputs
+    in a given precision carries, used for per-element fp32 tolerances.
+
+    Each output of the recurrence (Eq. 2 with readings R1, R4, R5 of ssd_oracle.c) expands
+    into a sum of products:
+      y_t[p]  = sum_n C_t[n] (prod_{s<=t} alpha_s h0[p][n]
+                              + sum_{s<=t} prod_{s<r<=t} alpha_r dt_s x_s[p] B_s[n]) + D x_t[p]
+    and every decay factor alpha = exp(dt*A) and every dt is positive, so the sum of the
+    absolute values of those products is the same recurrence run on |x|, |B|, |C|, |D| and
+    |h0|.  That is how it is evaluated here."""
+    def a(v):
+        return None if v is None else np.abs(np.asarray(v, dtype=np.float64))
+    return ssd_recurrence(a(x), dt, A, a(B), a(C), a(D), a(h0), nthreads=nthreads)
+
+
+def decode_step_mag(h_mag, conv_state, xbc, dt, A, D, conv_w, conv_b, act, G, N, nthreads=0):
+    """Term magnitudes of one decode step (see oracle_decode_step_mag in ssd_oracle.c).
+    ``h_mag`` [layers,b,H,P,N] float64 is updated in place (start it from |h|); conv_state
+    is the window BEFORE the step (call this ahead of decode_step).  Returns y_mag
+    [layers,b,H,P]."""
+    assert h_mag.dtype == np.float64 and h_mag.flags.c_contiguous
+    layers, b, H, P, Nn = h_mag.shape
+    assert Nn == N
+    k = conv_w.shape[2]
+    Dc = H * P + 2 * G * N
+    cs = _c(conv_state)
+    assert cs.shape == (layers, b, Dc, k - 1)
+    xbc, dt, A, D, conv_w, conv_b = map(_c, (xbc, dt, A, D, conv_w, conv_b))
+    ym = np.zeros((layers, b, H, P), np.float64)
+    _load().oracle_decode_step_mag(layers, b, H, P, N, G, k, int(act), _p(h_mag), _p(cs), _p(xbc), _p(dt),
+                                   _p(A), _p(D), _p(conv_w), _p(conv_b), _p(ym), int(nthreads))
+    return ym
 
 
 def dt_from_raw(dt_raw, dt_bias=None, dt_min=0.0, dt_max=float("inf")):

@@ -319,3 +319,66 @@ void oracle_dt_from_raw(size_t n, int H, const double* raw, const double* bias, 
         dt[i] = sp;
     }
 }
+
+/*
+ * Term magnitudes of one decode step, for per-element error bounds.  Every output of the
+ * step is a sum of products; an fp32 evaluation of it carries a rounding error of a few
+ * ulps of the SUM OF THE ABSOLUTE VALUES of those products, not of the output itself
+ * (which may cancel to near zero).  This function walks the same step as
+ * oracle_decode_step with each sum taken over absolute values:
+ *   window   = [conv_state[c][0..k-2], xbc[c]]      (read only: call before the value step)
+ *   m[c]     = sum_i |w[l][c][i] * window[i]| + |bias[l][c]|         the conv's terms
+ *   M[c]     = m[c] with no activation; |silu(v[c])| + m[c] with SiLU (its slope lies in
+ *              [-0.1, 1.1], so an error in the conv sum v moves the output by about as much)
+ *   hm[p][n] <- alpha*hm[p][n] + dt*Mx[p]*MB[n]    (hm starts from |h| and is updated in place)
+ *   ym[h][p] = sum_n MC[n]*hm[p][n] + |D|*Mx[p]
+ * Mx, MB, MC are the M of the x, B and C channels of the head's group.  Every magnitude
+ * bounds the absolute value of its output (triangle inequality), with equality when all
+ * inputs, weights and states are non-negative and no activation is applied.
+ */
+void oracle_decode_step_mag(int layers, int b, int H, int P, int N, int G, int kconv, int act,
+                            double* hm, const double* conv_state, const double* xbc, const double* dt,
+                            const double* A, const double* D, const double* conv_w,
+                            const double* conv_b, double* ym, int nthreads) {
+    set_threads(nthreads);
+    const int Dc = H * P + 2 * G * N, hpg = H / G, km1 = kconv - 1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int lb = 0; lb < layers * b; ++lb) {
+        const int l = lb / b, r = lb % b;
+        double* M = (double*)malloc(sizeof(double) * (size_t)Dc);
+        const double* cst = conv_state + ((size_t)l * b + r) * Dc * km1;
+        const double* xin = xbc + ((size_t)l * b + r) * Dc;
+        for (int c = 0; c < Dc; ++c) {
+            const double bias = conv_b[(size_t)l * Dc + c];
+            const double* w = conv_w + ((size_t)l * Dc + c) * kconv;
+            double v = bias, m = fabs(bias);
+            for (int i = 0; i < km1; ++i) {
+                v += w[i] * cst[(size_t)c * km1 + i];
+                m += fabs(w[i] * cst[(size_t)c * km1 + i]);
+            }
+            v += w[km1] * xin[c];
+            m += fabs(w[km1] * xin[c]);
+            M[c] = act == 1 ? fabs(v / (1.0 + exp(-v))) + m : m;
+        }
+        for (int hi = 0; hi < H; ++hi) {
+            const int g = hi / hpg;
+            const double d = dt[((size_t)l * b + r) * H + hi];
+            const double alpha = exp(d * A[(size_t)l * H + hi]);
+            const double* Mx = M + hi * P;
+            const double* MB = M + H * P + g * N;
+            const double* MC = M + H * P + G * N + g * N;
+            double* st = hm + ((((size_t)l * b + r) * H + hi) * P) * N;
+            double* yo = ym + (((size_t)l * b + r) * H + hi) * P;
+            for (int p = 0; p < P; ++p) {
+                double acc = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    const double v = alpha * st[p * N + n] + d * Mx[p] * MB[n];
+                    st[p * N + n] = v;
+                    acc += MC[n] * v;
+                }
+                yo[p] = acc + fabs(D[(size_t)l * H + hi]) * Mx[p];
+            }
+        }
+        free(M);
+    }
+}

@@ -308,3 +308,126 @@ def test_dt_from_raw_bias_per_head_and_clamp():
     np.testing.assert_allclose(got, np.broadcast_to([0.001, 0.01, 0.1, 1.0], raw.shape), rtol=1e-12)
     clamped = oracle.dt_from_raw(raw, bias, dt_min=0.005, dt_max=0.5)
     np.testing.assert_allclose(clamped[0, 0], [0.005, 0.01, 0.1, 0.5], rtol=1e-12)
+
+
+# ---------------------------------------------------------------- term magnitudes
+# The per-element fp32 tolerances scale with the sum of the absolute values of the products
+# behind each output.  These pins check that sum against an explicit enumeration of the
+# products (written here term by term, independently of the C recurrence) and against the
+# two properties that define it.
+
+def _enumerate_prefill_terms(x, dt, A, B, C, D, h0):
+    """Every product of the expanded recurrence for one sequence and one head (b = H = 1),
+    returned as lists of terms per output: y[t][p] and h_final[p][n]."""
+    x, dt, A, B, C, D, h0 = (np.asarray(v, np.float64) for v in (x, dt, A, B, C, D, h0))
+    T, P, N = x.shape[1], x.shape[3], B.shape[3]
+    a = dt[0, :, 0] * A[0]
+
+    def decay(s, t):  # prod of alpha_r for s < r <= t
+        return float(np.exp(a[s + 1:t + 1].sum()))
+
+    y_terms = [[[] for _ in range(P)] for _ in range(T)]
+    h_terms = [[[] for _ in range(N)] for _ in range(P)]
+    for t in range(T):
+        for p in range(P):
+            for n in range(N):
+                c = C[0, t, 0, n]
+                y_terms[t][p].append(c * decay(-1, t) * h0[0, 0, p, n])
+                for s in range(t + 1):
+                    y_terms[t][p].append(c * decay(s, t) * dt[0, s, 0] * x[0, s, 0, p] * B[0, s, 0, n])
+            y_terms[t][p].append(D[0] * x[0, t, 0, p])
+    for p in range(P):
+        for n in range(N):
+            h_terms[p][n].append(decay(-1, T - 1) * h0[0, 0, p, n])
+            for s in range(T):
+                h_terms[p][n].append(decay(s, T - 1) * dt[0, s, 0] * x[0, s, 0, p] * B[0, s, 0, n])
+    return y_terms, h_terms
+
+
+def test_prefill_magnitudes_enumerated():
+    """Catches: a magnitude taken of the wrong operand (C, B, x, h0 or D left signed), the
+    decay or dt dropped from a term, h0's term left out."""
+    x, dt, A, B, C, D, h0 = _tiny(b=1, T=5, H=1, P=2, N=3, seed=21)
+    D = np.array([-0.7])  # a signed skip weight, so |D| matters
+    ym, hm = oracle.ssd_magnitudes(x, dt, A, B, C, D, h0)
+    y_terms, h_terms = _enumerate_prefill_terms(x, dt, A, B, C, D, h0)
+    y_enum = np.array([[sum(abs(v) for v in y_terms[t][p]) for p in range(2)] for t in range(5)])
+    h_enum = np.array([[sum(abs(v) for v in h_terms[p][n]) for n in range(3)] for p in range(2)])
+    np.testing.assert_allclose(ym[0, :, 0, :], y_enum, rtol=1e-12, atol=0)
+    np.testing.assert_allclose(hm[0, 0], h_enum, rtol=1e-12, atol=0)
+    # and the enumeration is complete: its signed sums are the outputs themselves
+    y, hf = oracle.ssd_recurrence(x, dt, A, B, C, D, h0)
+    y_sum = np.array([[sum(y_terms[t][p]) for p in range(2)] for t in range(5)])
+    np.testing.assert_allclose(y[0, :, 0, :], y_sum, rtol=1e-12, atol=1e-14)
+
+
+def test_prefill_magnitudes_bound_and_equality():
+    """The magnitude bounds |output| (triangle inequality) and equals it when every input is
+    non-negative.  Catches a magnitude that is not a sum of absolute values."""
+    x, dt, A, B, C, D, h0 = _tiny(b=2, T=24, H=4, P=3, N=5, G=2, seed=22)
+    y, hf = oracle.ssd_recurrence(x, dt, A, B, C, D, h0)
+    ym, hm = oracle.ssd_magnitudes(x, dt, A, B, C, D, h0)
+    assert (np.abs(y) <= ym * (1 + 1e-12)).all() and (np.abs(hf) <= hm * (1 + 1e-12)).all()
+    assert (ym > np.abs(y) * (1 + 1e-6)).any()  # signs cancel somewhere
+    ax, aB, aC, ah = np.abs(x), np.abs(B), np.abs(C), np.abs(h0)
+    y2, hf2 = oracle.ssd_recurrence(ax, dt, A, aB, aC, D, ah)
+    ym2, hm2 = oracle.ssd_magnitudes(ax, dt, A, aB, aC, D, ah)
+    np.testing.assert_allclose(ym2, y2, rtol=1e-13, atol=0)
+    np.testing.assert_allclose(hm2, hf2, rtol=1e-13, atol=0)
+
+
+def test_decode_magnitudes_enumerated():
+    """One decode step with no activation, P = N = 1 and two conv taps, expanded into every
+    product: y = C (alpha h + dt x B) + D x with x, B, C each a sum of two tap products and a
+    bias.  Catches: a tap, the bias or the state term left out of the magnitude, |D| or the
+    conv weights left signed, the window read after the shift."""
+    rng = np.random.default_rng(5)
+    layers, b, H, P, N, G, k = 1, 1, 1, 1, 1, 1, 2
+    Dc = 3
+    h = rng.standard_normal((1, 1, 1, 1, 1))
+    cs = rng.standard_normal((1, 1, Dc, 1))
+    xbc = rng.standard_normal((1, 1, Dc))
+    dt = np.array([[[0.37]]])
+    A = np.array([[-1.9]])
+    D = np.array([[-0.6]])
+    w = rng.standard_normal((1, Dc, k))
+    bias = rng.standard_normal((1, Dc))
+    alpha = float(np.exp(dt[0, 0, 0] * A[0, 0]))
+    # tap products of each channel: [w0 * window0, w1 * current input, bias]
+    terms = [[w[0, c, 0] * cs[0, 0, c, 0], w[0, c, 1] * xbc[0, 0, c], bias[0, c]] for c in range(Dc)]
+    tx, tB, tC = terms
+    prods = [ci * alpha * h.item() for ci in tC]
+    prods += [ci * dt[0, 0, 0] * xi * bi for ci in tC for xi in tx for bi in tB]
+    prods += [D[0, 0] * xi for xi in tx]
+    hm = np.abs(h).copy()
+    ym = oracle.decode_step_mag(hm, cs, xbc, dt, A, D, w, bias, act=0, G=G, N=N)
+    assert abs(ym.item() - sum(abs(v) for v in prods)) <= 1e-12 * ym.item()
+    h_prods = [alpha * h.item()] + [dt[0, 0, 0] * xi * bi for xi in tx for bi in tB]
+    assert abs(hm.item() - sum(abs(v) for v in h_prods)) <= 1e-12 * hm.item()
+    # the enumeration is complete: its signed sum is the step's output
+    h2, cs2 = h.copy(), cs.copy()
+    y = oracle.decode_step(h2, cs2, xbc, dt, A, D, w, bias, act=0, G=G, N=N)
+    assert abs(y.item() - sum(prods)) <= 1e-12 * max(1.0, abs(y.item()))
+
+
+@pytest.mark.parametrize("act", [0, 1])
+def test_decode_magnitudes_bound_and_equality(act):
+    """|y| <= y_mag and |h| <= h_mag over several steps with either activation; with no
+    activation and every input, weight and state non-negative the two are equal."""
+    d = make_decode(layers=2, b=2, H=4, P=8, N=16, G=2, ring=3, seed=17)
+    h = d.h.astype(np.float64).copy()
+    cs = d.conv_state.astype(np.float64).copy()
+    hm = np.abs(h)
+    for s in range(3):
+        ym = oracle.decode_step_mag(hm, cs, d.xbc[s], d.dt[s], d.A, d.D, d.conv_w, d.conv_b, act=act, G=2, N=16)
+        y = oracle.decode_step(h, cs, d.xbc[s], d.dt[s], d.A, d.D, d.conv_w, d.conv_b, act=act, G=2, N=16)
+        assert (np.abs(y) <= ym * (1 + 1e-12)).all() and (np.abs(h) <= hm * (1 + 1e-12)).all()
+    if act == 0:
+        h = np.abs(d.h).astype(np.float64)
+        cs = np.abs(d.conv_state).astype(np.float64)
+        hm = h.copy()
+        w, bias, xbc = np.abs(d.conv_w), np.abs(d.conv_b), np.abs(d.xbc[0])
+        ym = oracle.decode_step_mag(hm, cs, xbc, d.dt[0], d.A, d.D, w, bias, act=0, G=2, N=16)
+        y = oracle.decode_step(h, cs, xbc, d.dt[0], d.A, d.D, w, bias, act=0, G=2, N=16)
+        np.testing.assert_allclose(ym, y, rtol=1e-13, atol=0)
+        np.testing.assert_allclose(hm, h, rtol=1e-13, atol=0)
