@@ -238,8 +238,10 @@ constexpr uint32_t kTmemSentinel = 0xFFFFFFFFu;
 __device__ __forceinline__ uint32_t tmem_alloc_cta(uint32_t* s_tmem, uint32_t cols, bool alloc_warp) {
     volatile uint32_t* slot = s_tmem;
     if (threadIdx.x == 0) *slot = kTmemSentinel;
+    __syncwarp();
     __syncthreads();
     if (alloc_warp) {
+        __syncwarp();
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
                      "r"(cols)
                      : "memory");
@@ -256,6 +258,7 @@ __device__ __forceinline__ uint32_t tmem_alloc_cta(uint32_t* s_tmem, uint32_t co
     return t;
 }
 __device__ __forceinline__ void group_bar(int id) {
+    __syncwarp();  // bar.sync is .aligned: each warp arrives converged
     asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kGroupThreads) : "memory");
 }
 __device__ __forceinline__ float ex2(float x) {
@@ -313,7 +316,10 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
         "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(bar)
         : "memory");
 }
-// TMEM <-> register moves.  tcgen05.ld writes its destination registers, and tcgen05.st
+// TMEM <-> register moves.  tcgen05.ld/st/wait are .sync.aligned: the whole warp must
+// execute them converged, so each macro first reconverges the warp (a store by a few
+// lanes or a lane-dependent select ahead of a move may otherwise leave it split).
+// tcgen05.ld writes its destination registers, and tcgen05.st
 // reads its source registers, asynchronously until the matching tcgen05.wait; each macro
 // issues the moves and the wait in ONE asm statement, so the compiler never sees the
 // registers as defined (or free) before the wait and cannot reuse, spill or read them
@@ -322,6 +328,8 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
 // load issues: an output of the first load, written asynchronously, can then never be the
 // register the second load reads its address from.
 #define SSD_TMEM_LD32_WAIT(taddr, r) \
+    do { \
+    __syncwarp(); \
     asm volatile( \
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t" \
         "tcgen05.wait::ld.sync.aligned;" \
@@ -331,8 +339,11 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
           "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), \
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31]) \
         : "r"(taddr) \
-        : "memory")
+        : "memory"); \
+    } while (0)
 #define SSD_TMEM_LD32x2_WAIT(ta, off, ra, rb) \
+    do { \
+    __syncwarp(); \
     asm volatile( \
         "{\n\t.reg .b32 tb;\n\tadd.u32 tb, %64, %65;\n\t" \
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t" \
@@ -349,8 +360,11 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
           "=r"(rb[24]), "=r"(rb[25]), "=r"(rb[26]), "=r"(rb[27]), "=r"(rb[28]), "=r"(rb[29]), "=r"(rb[30]), \
           "=r"(rb[31]) \
         : "r"(ta), "n"(off) \
-        : "memory")
+        : "memory"); \
+    } while (0)
 #define SSD_TMEM_LD16x2_WAIT(ta, off, ra, rb) \
+    do { \
+    __syncwarp(); \
     asm volatile( \
         "{\n\t.reg .b32 tb;\n\tadd.u32 tb, %32, %33;\n\t" \
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t" \
@@ -362,8 +376,11 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
           "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]), "=r"(rb[8]), "=r"(rb[9]), "=r"(rb[10]), "=r"(rb[11]), \
           "=r"(rb[12]), "=r"(rb[13]), "=r"(rb[14]), "=r"(rb[15]) \
         : "r"(ta), "n"(off) \
-        : "memory")
+        : "memory"); \
+    } while (0)
 #define SSD_TMEM_ST16x2_WAIT(ta, ra, tb, rb) \
+    do { \
+    __syncwarp(); \
     asm volatile( \
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17};\n\t" \
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%1], {%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};\n\t" \
@@ -374,7 +391,8 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
           "r"(ra[13]), "r"(ra[14]), "r"(ra[15]), "r"(rb[0]), "r"(rb[1]), "r"(rb[2]), "r"(rb[3]), \
           "r"(rb[4]), "r"(rb[5]), "r"(rb[6]), "r"(rb[7]), "r"(rb[8]), "r"(rb[9]), "r"(rb[10]), "r"(rb[11]), \
           "r"(rb[12]), "r"(rb[13]), "r"(rb[14]), "r"(rb[15]) \
-        : "memory")
+        : "memory"); \
+    } while (0)
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -782,8 +800,12 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 if (half == 0) {
                     s_cs[s * kBlk + r] = cs;
                     s_m[s * kBlk + r] = __log2f(dtv) - cs * kLog2e;   // -inf where dt = 0
-                    s_v[s * kBlk + r] = dexp<kDecay>(__expf(cend[q] - cs)) * dtv;  // cend[q]: end of j's group
-                    if (r < 4) s_cend[s * 4 + r] = cend[r];
+                    // cend[q] (the end of j's 32-token group) and, for lanes 0-3 of quadrant 0,
+                    // cend[lane], by selects: no dynamically indexed local array
+                    const float ce_q = q == 0 ? cend[0] : q == 1 ? cend[1] : q == 2 ? cend[2] : cend[3];
+                    const float ce_l = lane == 0 ? cend[0] : lane == 1 ? cend[1] : lane == 2 ? cend[2] : cend[3];
+                    s_v[s * kBlk + r] = dexp<kDecay>(__expf(ce_q - cs)) * dtv;
+                    if (r < 4) s_cend[s * 4 + r] = ce_l;
                 }
                 mbar_arrive(bar(BAR_PREP0 + s));
             }
@@ -860,9 +882,11 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     // The MMA lane has seen its final commit land and the producer its last loads; only
     // then is the TMEM released.
     tc_fence_before();
+    __syncwarp();
     __syncthreads();
     if (warp == 1 && tmem != kTmemSentinel) {
         tc_fence_after();
+        __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
 }
@@ -1078,9 +1102,11 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
     }
 
     tc_fence_before();
+    __syncwarp();
     __syncthreads();
     if (warp == 1 && tmem != kTmemSentinel) {
         tc_fence_after();
+        __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(SP::kTmemCols));
     }
 }
