@@ -309,7 +309,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--decode-steps", type=int, default=1024, help="timed decode steps at batch 1")
+    ap.add_argument("--decode-steps", type=int, default=4096,
+                    help="timed on-device decode steps per batch size (the cached-decode configuration's 4096)")
     ap.add_argument("--decode-batches", default="1,32")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-loop-compare", action="store_true",
@@ -531,6 +532,10 @@ def main():
         ablation = decay_precision_ablation(ssd, torch, dev)
 
     if rank == 0:
+        # the headline keys, then the roofline and a decode summary, so that a reader who
+        # keeps only the start of the line still has them; the details follow
+        decode_summary = {k: {"steps": v["steps"], "steps_per_s": v["steps_per_s"], "hbm_gbs_alg": v["hbm_gbs_alg"],
+                              "hbm_frac": v["hbm_frac"]} for k, v in decode.items()}
         line = {"metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -538,11 +543,12 @@ def main():
                            "G": PG, "chunk": PL, "global_batch": PB * world, "seq_len": PT,
                            "parallelism": "dp%d" % world,
                            "l2": "inputs larger than L2 (%.0f MB per step vs 126 MB)" % (pbytes / 1e6)},
+                "roofline": roofline, "decode_summary": decode_summary, "e2e": e2e, "cpu_baseline": cpu,
+                "gpu_launches": int(headline_launches),
                 "tokens_per_s": tokens_s, "step_ms": step_stats, "flops_per_step": flops, "chunk_executed": exec_L,
                 "tflops_at_requested_chunk": job_rate(flops_req, world, ms) / 1e12, "bytes_per_step": pbytes,
                 "hbm_gbs_alg": pbytes * world / (ms * 1e-3) / 1e9,
                 "tensor_frac": tflops / world / pk["bf16_tflops"],
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(headline_launches),
                 "gpu_launches_all_timed_regions": int(launches),
                 "clocks": clk, "decode": decode, "prefill_configs": other, "prefill_dt_raw": dt_raw_entry,
                 "decay_precision_ablation": ablation}
@@ -665,11 +671,11 @@ def bench_decode(ssd, torch, dev, stream, case, hf, b, args, clocks, barrier, ma
     ring = 256 if b == 1 else 32
     from ssd_inputs import make_decode_ring_device
     xbc, dt = make_decode_ring_device(ring, DL, b, DH, DP, DN, DG, dt_bias, seed=77, device=dev)
-    steps_per_launch = min(args.decode_steps if b == 1 else 64, 512)
+    steps_per_launch = min(args.decode_steps, 512 if b == 1 else 64)
     plan = ssd.DecodePlan(h, cst, xbc, dt, A, D, conv_w, conv_b, n_steps=steps_per_launch, G=DG)
     plan.launch()
     torch.cuda.synchronize()
-    launches_timed = max(1, (args.decode_steps if b == 1 else 128) // steps_per_launch)
+    launches_timed = max(1, args.decode_steps // steps_per_launch)
     barrier()
     n0 = ssd.launch_count()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
