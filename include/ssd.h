@@ -258,9 +258,11 @@ SSD_API int ssd_decode_step(int layers, int b, int H, int P, int N, int G, int k
  * scratch it needs (one 32-bit arrival counter per (layer, sequence, group)) lives in a
  * file-scope device array of SSD_DECODE_NOALLOC_MAX_COUNTERS counters (256 KiB) that
  * every GPU which loads the library keeps until the process exits; layers*b*G above
- * that limit returns SSD_ERR_INVALID_ARG.  The first call on a device looks up the
- * array's device address with that device current (cudaGetSymbolAddress), so make that
- * first call before any stream capture.  Each call clears the counters it uses
+ * that limit returns SSD_ERR_INVALID_ARG.  The first call in a CUDA context looks up the
+ * array's device address with that context current (cudaGetSymbolAddress) and caches it
+ * under the context's unique id, so make that first call before any stream capture; a
+ * context created later on the same device (after cudaDeviceReset, or a caller's own
+ * context) is looked up afresh, never served an address from a context that is gone.  Each call clears the counters it uses
  * (cudaMemsetAsync on `stream`) and calls no cudaMalloc, cudaFree or allocating
  * routine.  All calls on a device share the one array: calls that overlap on the GPU
  * (unordered streams) race on it and corrupt each other's conv windows.

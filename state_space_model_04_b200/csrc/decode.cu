@@ -16,6 +16,8 @@
 // finish (an arrival counter, no waiting) writes the shifted window back.
 #include "common.cuh"
 
+#include <cuda.h>
+
 #include <mutex>
 #include <vector>
 
@@ -299,22 +301,58 @@ static __device__ __align__(256) unsigned int g_noalloc_arrivals[SSD_DECODE_NOAL
 
 namespace ssd {
 
-// Device address and size of the scratch array on the current device.  The first call on
-// a device resolves the address with that device current and caches it.
+// Device address and size of the scratch array in the current context.  The address is
+// looked up (cudaGetSymbolAddress) the first time a context calls, with that context
+// current, and cached under the context's unique id: a context created later on the same
+// device -- after cudaDeviceReset, or a caller's own non-primary context -- has a new id
+// and gets its own lookup, so no call ever uses an address from a context that is gone.
+namespace {
+using PFN_ctxGetCurrent = CUresult (*)(CUcontext*);
+using PFN_ctxGetId = CUresult (*)(CUcontext, unsigned long long*);
+template <typename F>
+F driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<F>(p);
+}
+// unique id of the current context (0 if none is current or the driver cannot say)
+unsigned long long current_context_id() {
+    static PFN_ctxGetCurrent get_cur = driver_fn<PFN_ctxGetCurrent>("cuCtxGetCurrent");
+    static PFN_ctxGetId get_id = driver_fn<PFN_ctxGetId>("cuCtxGetId");
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (!get_cur || !get_id || get_cur(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+}  // namespace
+
 int decode_noalloc_scratch(void** ptr, size_t* bytes) {
-    constexpr int kMaxDevices = 64;
+    constexpr int kSlots = 64;
     static std::mutex mu;
-    static void* addr[kMaxDevices] = {};
-    int dev = 0;
-    SSD_CUDA_TRY(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= kMaxDevices) return set_error(SSD_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kMaxDevices - 1);
+    static unsigned long long ids[kSlots] = {};
+    static void* addrs[kSlots] = {};
+    static int next = 0;
+    // the lookup also makes the device's primary context current if nothing is yet
+    void* p = nullptr;
+    unsigned long long id = current_context_id();
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void* p = nullptr;
-        SSD_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_arrivals));
-        addr[dev] = p;
+    if (id != 0)
+        for (int i = 0; i < kSlots; ++i)
+            if (ids[i] == id) {
+                *ptr = addrs[i];
+                *bytes = sizeof(g_noalloc_arrivals);
+                return SSD_OK;
+            }
+    SSD_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_arrivals));
+    if (id == 0) id = current_context_id();  // the lookup created the primary context
+    if (id != 0) {
+        ids[next] = id;
+        addrs[next] = p;
+        next = (next + 1) % kSlots;
     }
-    *ptr = addr[dev];
+    *ptr = p;
     *bytes = sizeof(g_noalloc_arrivals);
     return SSD_OK;
 }
