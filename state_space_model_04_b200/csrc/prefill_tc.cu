@@ -16,23 +16,35 @@
 // as two such blocks with the state handed between them -- the same dual form over a
 // shorter segment, identical in exact arithmetic.
 //
+// Only the state recurrence is sequential; the dual form of a block needs nothing from the
+// blocks before it.  The kernel therefore runs two pipelines that meet only at the output:
+// the scores path (C B^T -> P -> P X) runs up to a block ahead of the state path
+// (w o X -> S -> H -> C H^T), each with its own MMA-issuing warp, and every TMEM buffer the
+// scores path needs is doubled so it never waits for the block before.
+//
 //   warp 0       TMA producer: C and B (two 64-column 128B-swizzled boxes each) into a
-//                2-slot ring, X into a 3-slot ring (slot k % 3 later holds y of block k)
-//   warp 1       TMEM owner and MMA issuer (one lane).  Iteration k:
-//                  Y(k)      = P(k) X(k)      (M=128 i, N=64 p,  K=128 j)  TS, P in TMEM
-//                  CB(k+1)   = C B^T          (M=128 i, N=128 j, K=128 n)  SS
-//                  Yst(k+1)  = C H^T          (M=128 i, N=64 p,  K=128 n)  SS
-//                  S(k+1)^T  = B^T (w o X)    (M=128 n, N=64 p,  K=128 j)  SS
-//                so C and B of a block are dead within one iteration and the next
-//                block's loads run a full iteration ahead of their use.
-//   warps 2-9    "scores" group (2 warps per TMEM lane quadrant): P = bf16(CB o L),
-//                written back into TMEM as the A operand of P X; y = Y + exp(cs_i) Yst
-//                into a swizzled shared tile (the block's dead X slot)
-//   warps 10-17  "state" group (2 warps per quadrant): prefix sums of dt*A, the decay
-//                arrays, w o X into shared memory, H <- exp(cs_last) H + S (fp32
-//                registers) with its bf16 copy for C H^T
-//   warp 18      y store: one TMA tensor store per block, then the X slot goes back to
+//                2-slot ring, X into a 3-slot ring
+//   warp 1       TMEM owner; issues the scores path (one elected lane):
+//                  CB(k)     = C B^T          (M=128 i, N=128 j, K=128 n)  SS -> CB/P buffer k&1
+//                  Y(k)      = P(k) X(k)      (M=128 i, N=64 p,  K=128 j)  TS, P in buffer k&1
+//                in the order CB(k+1), Y(k), so C B^T runs one block ahead
+//   warp 2       issues the state path:
+//                  S(k)^T    = B^T (w o X)    (M=128 n, N=64 p,  K=128 j)  SS
+//                  Yst(k)    = C H(k)^T       (M=128 i, N=64 p,  K=128 n)  SS -> buffer k&1
+//   warps 3-10   "scores" group (2 warps per TMEM lane quadrant): P = bf16(CB o L) written
+//                back IN PLACE over the C B^T columns it was computed from (chunk c of 32
+//                score columns -> the first 16 of its 32 columns, bf16 pairs), the A
+//                operand of P X; then for the previous block y = Y + exp(cs_i) Yst into a
+//                swizzled shared tile (the block's X slot, dead by then)
+//   warps 11-18  "state" group (2 warps per quadrant): w o X into shared memory, H <-
+//                exp(cs_last) H + S in fp32 registers, its bf16 copy H^T for C H^T
+//   warp 19      y store: one TMA tensor store per block, then the X slot goes back to
 //                the producer
+//   warp 20      "prep": prefix sums of dt*A and every per-token decay term of a block (the
+//                scores group's and the state group's), two blocks ahead of their use
+//
+// A warp whose TMEM lane quadrant is q is warp q (mod 4): warps 3-10 and 11-18 map onto
+// the quadrants 3, 0, 1, 2, 3, 0, 1, 2.
 //
 // Decay arithmetic.  Below the 32x32 diagonal sub-blocks the decay factorises exactly
 // as exp(cs_i - cs_e) * exp(cs_e - cs_j) with e the last token of j's 32-token group
@@ -58,7 +70,10 @@ constexpr int kBlk = 128;    // tokens per block = MMA M
 constexpr int kP = 64;       // head dim
 constexpr int kN = 128;      // state size
 constexpr int kGroupThreads = 256;  // threads per epilogue group
-constexpr int kThreads = 64 + 2 * kGroupThreads + 32;  // + the y-store warp
+constexpr int kWarpScores = 3, kWarpState = 11;
+constexpr int kWarpStore = kWarpState + 8;         // the y-store warp
+constexpr int kWarpPrep = kWarpStore + 1;          // the decay-term warp
+constexpr int kThreads = 32 * (kWarpPrep + 1);     // 21 warps
 constexpr float kLog2e = 1.4426950408889634f;
 
 // shared memory map (bytes from a 1024-aligned base)
@@ -71,41 +86,53 @@ constexpr uint32_t kXRing = 2 * kCBSlot;             // 3 X slots of one region;
 constexpr uint32_t kXs = kXRing + 3 * kRegion;       // w o X
 constexpr uint32_t kSH = kXs + kRegion;              // bf16 H^T [n][p]
 constexpr uint32_t kSmall = kSH + kRegion;           // barriers and per-token scalars
-constexpr uint32_t kSmallBytes = 4096;
+constexpr uint32_t kSmallBytes = 5120;
 constexpr uint32_t kSmemBytes = kSmall + kSmallBytes;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kSmemBytes <= 232448 - 1024, "shared memory budget (1 KB of static shared memory beside it)");
 
 // TMEM columns (512 x 128 lanes x 32 bit)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColCB = 0;      // fp32 C B^T (128 columns)
-constexpr uint32_t kColP = 128;     // bf16 scores, 2 per column (64 columns)
-constexpr uint32_t kColS = 192;     // fp32 S^T (64 columns)
-constexpr uint32_t kColY = 256;     // two 64-column Y buffers
-constexpr uint32_t kColYst = 384;   // two 64-column C H^T buffers
+constexpr uint32_t kColCBP = 0;     // two 128-column buffers: fp32 C B^T, then bf16 P in place
+constexpr uint32_t kColY = 256;     // fp32 Y (64 columns)
+constexpr uint32_t kColYst = 320;   // two 64-column C H^T buffers
+constexpr uint32_t kColS = 448;     // fp32 S^T (64 columns)
+static_assert(kColS + 64 == kTmemCols, "TMEM map");
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
-// barrier indices in the small area
+// barrier indices in the small area; [n] = n barriers indexed by block (k & 1, or k % 3)
 enum {
-    BAR_FULLCB = 0,   // [2] C,B landed
-    BAR_EMPTYCB = 2,  // [2] C,B slot released by the MMAs
-    BAR_FULLX = 4,    // [3] X landed
-    BAR_EMPTYX = 7,   // [3] X slot released (its y tile has been read by the TMA store)
-    BAR_CBFULL = 10,  // C B^T accumulated
-    BAR_CBFREE,       // scores group has read C B^T            (256 arrivals)
-    BAR_XS,           // state group has written w o X          (256)
-    BAR_ACCS,         // S^T accumulated (and w o X read)
-    BAR_SFREE,        // state group has read S^T               (256)
-    BAR_YSTDONE,      // C H^T accumulated (and bf16 H read)
-    BAR_H,            // state group has written bf16 H         (256)
-    BAR_SCORES,       // scores group has written P             (256)
-    BAR_G2DONE,       // P X accumulated (and P read)
-    BAR_YFREE0,       // [2] scores group has read Y and C H^T of the slot (256)
-    BAR_PREP0 = BAR_YFREE0 + 2,  // [2] state group has published a block's decay arrays (256)
-    BAR_YSTAGED = BAR_PREP0 + 2,  // [3] scores group has written the y tile into X slot (256)
-    BAR_DONE = BAR_YSTAGED + 3,
+    BAR_FULLCB = 0,    // [2] C,B landed (TMA transaction bytes)
+    BAR_EMPTYCB = 2,   // [2] C,B slot free: C B^T (issuer 1) and S, C H^T (issuer 2) done  (2 arrivals)
+    BAR_FULLX = 4,     // [3] X landed
+    BAR_EMPTYX = 7,    // [3] X slot free: its y tile has been read out by the TMA store
+    BAR_CBFULL = 10,   // [2] C B^T accumulated in CB/P buffer k & 1
+    BAR_PREADY = 12,   // [2] scores group wrote P over it                              (256)
+    BAR_PXDONE = 14,   // [2] Y = P X accumulated: the CB/P buffer is free again
+    BAR_YFREE = 16,    // scores group read Y                                            (256)
+    BAR_PREP = 17,     // [2] the prep warp published a block's decay terms              (1)
+    BAR_XSREADY = 19,  // state group wrote w o X                                        (256)
+    BAR_SDONE = 20,    // S^T accumulated (w o X read)
+    BAR_SFREE = 21,    // state group read S^T                                           (256)
+    BAR_HREADY = 22,   // state group wrote bf16 H^T                                     (256)
+    BAR_YSTDONE = 23,  // [2] C H^T accumulated (H^T read)
+    BAR_YSTFREE = 25,  // [2] scores group read C H^T                                    (256)
+    BAR_YSTAGED = 27,  // [3] scores group wrote block k's y tile into X slot k % 3          (256)
+    BAR_ARRFREE = 30,  // [2] a block's decay terms read: scores and state warps      (16 warps)
+    BAR_DONE1 = 32,    // every MMA of issuer 1 complete (teardown)
+    BAR_DONE2 = 33,    // every MMA of issuer 2 complete (teardown)
     BAR_COUNT
 };
+static_assert(BAR_COUNT * 8 <= 512, "barriers fit ahead of the per-token arrays");
+__host__ __device__ constexpr uint32_t bar_count(int i) {
+    return (i == BAR_EMPTYCB || i == BAR_EMPTYCB + 1) ? 2u
+           : (i == BAR_ARRFREE || i == BAR_ARRFREE + 1) ? 16u
+           : (i == BAR_PREADY || i == BAR_PREADY + 1 || i == BAR_YFREE ||
+              i == BAR_XSREADY || i == BAR_SFREE || i == BAR_HREADY || i == BAR_YSTFREE || i == BAR_YSTFREE + 1 ||
+              (i >= BAR_YSTAGED && i < BAR_YSTAGED + 3))
+               ? (uint32_t)kGroupThreads
+               : 1u;
+}
 
 struct TcParams {
     CUtensorMap tm_x;
@@ -179,10 +206,11 @@ __device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 // Bounded wait for the phase with `parity` to complete.  Returns false (and makes every
-// other role give up) if the CTA is aborting or the limit expires.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status, int where) {
-    if (mbar_try(bar, parity)) return true;
+// other role give up) if the CTA is aborting or the limit expires.  The first test is
+// inline; the waiting loop is one out-of-line copy shared by every call site, which keeps
+// the kernel's hot code small (instruction fetch, not arithmetic, bounds the busy warps).
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                            int where) {
     const unsigned long long t0 = globaltimer();
     while (true) {
         if (mbar_try_sleep(bar, parity)) return true;
@@ -193,6 +221,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             return false;
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                          int where) {
+    if (mbar_try(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, abort_flag, status, where);
 }
 // The same, voted across the warp so that warp-collective tcgen05 instructions after it
 // are executed by all lanes or by none.
@@ -362,7 +395,9 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
         : "r"(ta), "n"(off) \
         : "memory"); \
     } while (0)
-#define SSD_TMEM_LD16x2_WAIT(ta, off, ra, rb) \
+#define SSD_TMEM_LD16x2_WAIT(ta, off, ra, rb) SSD_TMEM_LD16x2_WAIT_(ta, off, ra, rb, "n")
+#define SSD_TMEM_LD16x2_WAIT_R(ta, off, ra, rb) SSD_TMEM_LD16x2_WAIT_(ta, off, ra, rb, "r")
+#define SSD_TMEM_LD16x2_WAIT_(ta, off, ra, rb, kind) \
     do { \
     __syncwarp(); \
     asm volatile( \
@@ -375,7 +410,19 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
           "=r"(ra[14]), "=r"(ra[15]), "=r"(rb[0]), "=r"(rb[1]), "=r"(rb[2]), "=r"(rb[3]), "=r"(rb[4]), \
           "=r"(rb[5]), "=r"(rb[6]), "=r"(rb[7]), "=r"(rb[8]), "=r"(rb[9]), "=r"(rb[10]), "=r"(rb[11]), \
           "=r"(rb[12]), "=r"(rb[13]), "=r"(rb[14]), "=r"(rb[15]) \
-        : "r"(ta), "n"(off) \
+        : "r"(ta), kind(off) \
+        : "memory"); \
+    } while (0)
+#define SSD_TMEM_ST16_WAIT(ta, ra) \
+    do { \
+    __syncwarp(); \
+    asm volatile( \
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t" \
+        "tcgen05.wait::st.sync.aligned;" \
+        : \
+        : "r"(ta), "r"(ra[0]), "r"(ra[1]), "r"(ra[2]), "r"(ra[3]), "r"(ra[4]), "r"(ra[5]), "r"(ra[6]), \
+          "r"(ra[7]), "r"(ra[8]), "r"(ra[9]), "r"(ra[10]), "r"(ra[11]), "r"(ra[12]), "r"(ra[13]), "r"(ra[14]), \
+          "r"(ra[15]) \
         : "memory"); \
     } while (0)
 #define SSD_TMEM_ST16x2_WAIT(ta, ra, tb, rb) \
@@ -454,15 +501,15 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 
     uint8_t* small = smem + kSmall;
     uint64_t* bars = reinterpret_cast<uint64_t*>(small);              // BAR_COUNT barriers
-    // per-token decay arrays of a block, published by the state group for the scores group
-    float* s_m = reinterpret_cast<float*>(small + 256);               // [2][128] log2(dt_j) - cs_j log2e
+    // per-token decay terms of a block (two slots), published by the prep warp
+    float* s_m = reinterpret_cast<float*>(small + 512);               // [2][128] log2(dt_j) - cs_j log2e
     float* s_v = s_m + 2 * kBlk;                                      // [2][128] exp(cs_e - cs_j) dt_j
     float* s_cs = s_v + 2 * kBlk;                                     // [2][128] cs_i
-    float* s_cend = s_cs + 2 * kBlk;                                  // [2][4] cs at the end of each 32-token group
-    float* s_ytot = s_cend + 8;                                       // [2][4] state-group quadrant sums
-    volatile int* s_abort = reinterpret_cast<volatile int*>(s_ytot + 8);
-    volatile int* s_ystop = s_abort + 1;                              // [2]
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_ytot + 16);
+    float* s_w = s_cs + 2 * kBlk;                                     // [2][128] exp(cs_last - cs_j) dt_j
+    float* s_cend = s_w + 2 * kBlk;                                   // [2][4] cs at the end of each 32-token group
+    float* s_cslast = s_cend + 8;                                     // [2] the block's total log decay
+    volatile int* s_abort = reinterpret_cast<volatile int*>(s_cslast + 2);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(s_cslast + 4);
 
     const uint32_t sbase = smem_u32(smem);
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -470,15 +517,9 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     if (threadIdx.x == 0) {
         const bool misaligned = (sbase & 1023u) != 0;  // swizzled layouts need a 1024-byte base
         if (misaligned) atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (1 << 8));
-        for (int i = 0; i < BAR_COUNT; ++i) {
-            const bool group = (i == BAR_CBFREE || i == BAR_XS || i == BAR_SFREE || i == BAR_H ||
-                                i == BAR_SCORES || i == BAR_YFREE0 || i == BAR_YFREE0 + 1 || i == BAR_PREP0 ||
-                                i == BAR_PREP0 + 1 || (i >= BAR_YSTAGED && i < BAR_YSTAGED + 3));
-            mbar_init(bar(i), group ? kGroupThreads : 1);
-        }
+        for (int i = 0; i < BAR_COUNT; ++i) mbar_init(bar(i), bar_count(i));
         *s_abort = misaligned ? 1 : 0;
         s_wait_ns = prm.wait_ns;
-        s_ystop[0] = s_ystop[1] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     const uint32_t tmem = tmem_alloc_cta(s_tmem, kTmemCols, warp == 1);  // warp 1 owns the TMEM
@@ -520,117 +561,136 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 if (u >= 0) mbar_drain(bar(BAR_FULLX + u % 3), (u / 3) & 1);
         }
     } else if (warp == 1) {
-        // ================================================================ MMA issuer
-        // The whole warp runs this loop (operands stay warp-uniform); one elected lane
-        // issues each tcgen05 instruction.
+        // ================================================================ issuer 1: scores path
+        // The whole warp runs this loop (operands stay warp-uniform); one elected lane issues
+        // each tcgen05 instruction.
         constexpr uint32_t id_cb = idesc_bf16(128, 128, 0, 0);   // A C (K-major), B B (K-major)
-        constexpr uint32_t id_s = idesc_bf16(128, 64, 1, 1);     // A B^T (MN-major), B w o X (MN-major)
         constexpr uint32_t id_y = idesc_bf16(128, 64, 0, 1);     // A P (TMEM), B X (MN-major)
+        auto wt = [&](int b, uint32_t parity, int where) {
+            return warp_wait(bar(b), parity, s_abort, prm.status, where);
+        };
+        auto issue_cb = [&](int k) {  // C B^T of block k (C, B in ring slot k & 1) into CB/P buffer k & 1
+            const uint32_t slot = sbase + (k & 1) * kCBSlot;
+            const uint64_t dC = sdesc(slot + kSlotC, 16, 1024), dB = sdesc(slot + kSlotB, 16, 1024);
+            // a K step of 16 advances only the 16-byte address field of a K-major descriptor.
+            // The K loops stay rolled: each tcgen05.mma site costs a few hundred bytes of code,
+            // and instruction fetch, not issue rate, limits these warps
+#pragma unroll 1
+            for (int kk = 0; kk < kN / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * (kRegion >> 4) + (kk & 3) * 2;
+                mma_ss_w(tmem + kColCBP + (k & 1) * 128, dC + off, dB + off, id_cb, kk > 0);
+            }
+            mma_commit_w(bar(BAR_CBFULL + (k & 1)));
+            mma_commit_w(bar(BAR_EMPTYCB + (k & 1)));
+        };
+        auto issue_y = [&](int k) {  // Y = P_k X_k; P chunk c (K steps 2c, 2c+1) sits at column 32c
+            const uint64_t dX = sdesc(sbase + kXRing + (k % 3) * kRegion, kRegion, 1024);
+            const uint32_t pbuf = tmem + kColCBP + (k & 1) * 128;
+#pragma unroll 1
+            for (int kk = 0; kk < kBlk / 16; ++kk)
+                mma_ts_w(tmem + kColY, pbuf + (kk >> 1) * 32 + (kk & 1) * 8, dX + kk * 128, id_y, kk > 0);
+            mma_commit_w(bar(BAR_PXDONE + (k & 1)));
+        };
+        bool ok = __all_sync(0xffffffffu, !*s_abort);
+        if (ok && nblk > 0) {
+            ok = wt(BAR_FULLCB, 0, 3);
+            if (ok) { tc_fence_after(); issue_cb(0); }
+        }
+        for (int k = 0; k < nblk && ok; ++k) {
+            // C B^T of the next block first: the scores group's longest lead.  Its buffer was
+            // last read by P X of block k - 1.
+            if (k + 1 < nblk) {
+                ok = wt(BAR_FULLCB + ((k + 1) & 1), ((k + 1) >> 1) & 1, 7) &&
+                     (k < 1 || wt(BAR_PXDONE + ((k + 1) & 1), ((k - 1) >> 1) & 1, 4));
+                if (!ok) break;
+                tc_fence_after();
+                issue_cb(k + 1);
+            }
+            // Y of block k: P written, X landed, and the scores group done reading Y of block k - 1
+            ok = wt(BAR_PREADY + (k & 1), (k >> 1) & 1, 9) && wt(BAR_FULLX + k % 3, (k / 3) & 1, 8) &&
+                 (k < 1 || wt(BAR_YFREE, (k - 1) & 1, 10));
+            if (!ok) break;
+            tc_fence_after();
+            issue_y(k);
+        }
+        // every MMA and commit issued above completes before the TMEM is released
+        mma_commit_w(bar(BAR_DONE1));
+        mbar_drain(bar(BAR_DONE1), 0);
+    } else if (warp == 2) {
+        // ================================================================ issuer 2: state path
+        constexpr uint32_t id_s = idesc_bf16(128, 64, 1, 1);     // A B^T (MN-major), B w o X (MN-major)
         constexpr uint32_t id_yst = idesc_bf16(128, 64, 0, 1);   // A C (K-major), B H^T (MN-major)
         auto wt = [&](int b, uint32_t parity, int where) {
             return warp_wait(bar(b), parity, s_abort, prm.status, where);
         };
-        auto issue_cb = [&](int u) {  // C B^T of block u (C, B in ring slot u & 1)
-            const uint32_t slot = sbase + (u & 1) * kCBSlot;
-            const uint64_t dC = sdesc(slot + kSlotC, 16, 1024), dB = sdesc(slot + kSlotB, 16, 1024);
-            // a K step of 16 advances only the 16-byte address field of a K-major descriptor
-#pragma unroll
-            for (int k = 0; k < kN / 16; ++k) {
-                const uint32_t off = (k >> 2) * (kRegion >> 4) + (k & 3) * 2;
-                mma_ss_w(tmem + kColCB, dC + off, dB + off, id_cb, k > 0);
-            }
-            mma_commit_w(bar(BAR_CBFULL));
-        };
-        auto issue_yst = [&](int u) {  // C H_u^T
-            const uint32_t slot = sbase + (u & 1) * kCBSlot;
-            const uint64_t dC = sdesc(slot + kSlotC, 16, 1024), dH = sdesc(sbase + kSH, kRegion, 1024);
-#pragma unroll
-            for (int k = 0; k < kN / 16; ++k) {
-                const uint32_t off = (k >> 2) * (kRegion >> 4) + (k & 3) * 2;
-                mma_ss_w(tmem + kColYst + (u & 1) * 64, dC + off, dH + k * 128, id_yst, k > 0);  // MN step: 16 rows
-            }
-            mma_commit_w(bar(BAR_YSTDONE));
-        };
-        auto issue_state = [&](int u) {  // S_u^T = B^T (w o X); then C, B of block u are dead
-            const uint32_t slot = sbase + (u & 1) * kCBSlot;
+        auto issue_s = [&](int k) {  // S_k^T = B^T (w o X)
+            const uint32_t slot = sbase + (k & 1) * kCBSlot;
             const uint64_t dBt = sdesc(slot + kSlotB, kRegion, 1024), dXs = sdesc(sbase + kXs, kRegion, 1024);
-#pragma unroll
-            for (int k = 0; k < kBlk / 16; ++k) mma_ss_w(tmem + kColS, dBt + k * 128, dXs + k * 128, id_s, k > 0);
-            mma_commit_w(bar(BAR_ACCS));
-            mma_commit_w(bar(BAR_EMPTYCB + (u & 1)));
+#pragma unroll 1
+            for (int kk = 0; kk < kBlk / 16; ++kk) mma_ss_w(tmem + kColS, dBt + kk * 128, dXs + kk * 128, id_s, kk > 0);
+            mma_commit_w(bar(BAR_SDONE));
         };
-        auto issue_y = [&](int k) {  // Y_k = P_k X_k; then X of block k is dead
-            const uint64_t dX = sdesc(sbase + kXRing + (k % 3) * kRegion, kRegion, 1024);
-#pragma unroll
-            for (int kk = 0; kk < kBlk / 16; ++kk)
-                mma_ts_w(tmem + kColY + (k & 1) * 64, tmem + kColP + kk * 8, dX + kk * 128, id_y, kk > 0);
-            mma_commit_w(bar(BAR_G2DONE));
+        auto issue_yst = [&](int k) {  // C H_k^T into buffer k & 1; then C, B of block k are dead
+            const uint32_t slot = sbase + (k & 1) * kCBSlot;
+            const uint64_t dC = sdesc(slot + kSlotC, 16, 1024), dH = sdesc(sbase + kSH, kRegion, 1024);
+#pragma unroll 1
+            for (int kk = 0; kk < kN / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * (kRegion >> 4) + (kk & 3) * 2;
+                mma_ss_w(tmem + kColYst + (k & 1) * 64, dC + off, dH + kk * 128, id_yst, kk > 0);  // MN step: 16 rows
+            }
+            mma_commit_w(bar(BAR_YSTDONE + (k & 1)));
+            mma_commit_w(bar(BAR_EMPTYCB + (k & 1)));
         };
         bool ok = __all_sync(0xffffffffu, !*s_abort);
-        if (ok) {
-            // block 0: C B^T, C H_0^T, S_0
-            ok = wt(BAR_FULLCB, 0, 3);
-            if (ok) { tc_fence_after(); issue_cb(0); ok = wt(BAR_H, 0, 5); }
-            if (ok) { tc_fence_after(); issue_yst(0); ok = wt(BAR_XS, 0, 6); }
-            if (ok) { tc_fence_after(); issue_state(0); }
-            // iteration k: C B^T(k+1) first (the scores group's longest lead), then P X (k),
-            // C H^T (k+1) and S(k+1)
-            for (int k = 0; k < nblk && ok; ++k) {
-                if (k + 1 < nblk) {
-                    ok = wt(BAR_FULLCB + ((k + 1) & 1), ((k + 1) >> 1) & 1, 7) && wt(BAR_CBFREE, k & 1, 4);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_cb(k + 1);
-                }
-                // Y and C H^T buffers k & 1 were last read for block k - 2
-                ok = wt(BAR_FULLX + k % 3, (k / 3) & 1, 8) && wt(BAR_SCORES, k & 1, 9) &&
-                     (k < 2 || wt(BAR_YFREE0 + (k & 1), ((k - 2) >> 1) & 1, 10));
-                if (!ok) break;
-                tc_fence_after();
-                issue_y(k);
-                if (k + 1 < nblk) {
-                    // C H^T buffer (k+1) & 1 was last read (with Y) for block k - 1
-                    ok = wt(BAR_H, (k + 1) & 1, 5) &&
-                         (k < 1 || wt(BAR_YFREE0 + ((k + 1) & 1), ((k - 1) >> 1) & 1, 19));
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_yst(k + 1);
-                    ok = wt(BAR_XS, (k + 1) & 1, 6) && wt(BAR_SFREE, k & 1, 11);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_state(k + 1);
-                }
-            }
-            // every MMA and commit issued above completes before the TMEM is released
-            mma_commit_w(bar(BAR_DONE));
-            mbar_drain(bar(BAR_DONE), 0);
+        for (int k = 0; k < nblk && ok; ++k) {
+            // S of block k: C,B landed, w o X written, and S of block k - 1 read
+            ok = wt(BAR_FULLCB + (k & 1), (k >> 1) & 1, 21) && wt(BAR_XSREADY, k & 1, 22) &&
+                 (k < 1 || wt(BAR_SFREE, (k - 1) & 1, 23));
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(k);
+            // C H^T of block k: H^T of the state entering block k written, and its buffer read
+            // by the scores group for block k - 2
+            ok = wt(BAR_HREADY, k & 1, 24) && (k < 2 || wt(BAR_YSTFREE + (k & 1), ((k - 2) >> 1) & 1, 25));
+            if (!ok) break;
+            tc_fence_after();
+            issue_yst(k);
         }
-    } else if (warp < 10) {
+        mma_commit_w(bar(BAR_DONE2));
+        mbar_drain(bar(BAR_DONE2), 0);
+    } else if (warp < kWarpState) {
         // ================================================================ scores group
-        const int q = warp & 3, half = (warp - 2) >> 2;
+        const int q = warp & 3, half = (warp - kWarpScores) >> 2;
         const int r = q * 32 + lane;  // token row i (and column index j for the per-token arrays)
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
         const float Dh = prm.D[hd];
         const int p0 = half * 32;  // this warp's 32 of the 64 p columns of the output
         // y(k) = Y(k) + exp(cs_i) Yst(k) for row r, columns [p0, p0 + 32), into the swizzled
-        // y tile in X slot k % 3 (X(k) is dead once P X of block k is done, which every
-        // caller has waited for); the store warp writes the tile out with one TMA store.
+        // y tile in X slot k % 3: X(k) is dead once P X of block k is done and C H^T of block
+        // k is done (the state group read X(k) for w o X before it published H^T(k), which
+        // C H^T waited for).  The store warp writes the tile out with one TMA store.
         // exp(cs_i) is carried in a register: by now the state group may have republished
-        // the per-token arrays of block k's slot.
+        // the arrays of block k's slot.
         auto store_y = [&](int k, float ei) {
+            bool ok = warp_wait(bar(BAR_PXDONE + (k & 1)), (k >> 1) & 1, s_abort, prm.status, 12);
+            if (ok) ok = warp_wait(bar(BAR_YSTDONE + (k & 1)), (k >> 1) & 1, s_abort, prm.status, 18);
+            if (!ok) return false;
             tc_fence_after();
             uint32_t yp[16];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t ry[16], rs[16];
-                SSD_TMEM_LD16x2_WAIT(tmem + lane_addr + kColY + (k & 1) * 64 + p0 + hh * 16, kColYst - kColY, ry, rs);
+                const uint32_t ta = tmem + lane_addr + kColY + p0 + hh * 16;
+                const uint32_t off = kColYst + (k & 1) * 64 - kColY;
+                SSD_TMEM_LD16x2_WAIT_R(ta, off, ry, rs);
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     yp[hh * 8 + j] = pack_bf16(fmaf(ei, __uint_as_float(rs[2 * j]), __uint_as_float(ry[2 * j])),
                                                fmaf(ei, __uint_as_float(rs[2 * j + 1]), __uint_as_float(ry[2 * j + 1])));
             }
             tc_fence_before();
-            mbar_arrive(bar(BAR_YFREE0 + (k & 1)));
+            mbar_arrive(bar(BAR_YFREE));
+            mbar_arrive(bar(BAR_YSTFREE + (k & 1)));
             uint8_t* dst = smem + kXRing + (k % 3) * kRegion;
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4)
@@ -644,38 +704,29 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         float ei_prev = 0.f;  // exp(cs_i) of the previous block
         for (int u = 0; u < nblk; ++u) {
             const int s = u & 1;
+            const uint32_t buf = tmem + lane_addr + kColCBP + s * 128;
             float ei_cur = 0.f;
             // the state group publishes cs, the chunk ends and the per-column decay terms
-            if (live) live = warp_wait(bar(BAR_PREP0 + s), (u >> 1) & 1, s_abort, prm.status, 17);
-            // ---- P = bf16(CB o L) for this warp's chunks {half, half + 2} of row r
-            uint32_t pk[2][16];
-            if (live) live = warp_wait(bar(BAR_CBFULL), u & 1, s_abort, prm.status, 11);
+            if (live) live = warp_wait(bar(BAR_PREP + s), (u >> 1) & 1, s_abort, prm.status, 17);
+            if (live) live = warp_wait(bar(BAR_CBFULL + s), (u >> 1) & 1, s_abort, prm.status, 11);
             if (live) {
+                // ---- P = bf16(CB o L) for this warp's chunks {half, half + 2} of row r,
+                //      written over the first 16 of each chunk's 32 columns
                 tc_fence_after();
                 const float* vs = s_v + s * kBlk;
                 const float* ms = s_m + s * kBlk;
                 const float cs = s_cs[s * kBlk + r];
                 const float csl = cs * kLog2e;
                 ei_cur = dexp<kDecay>(__expf(cs));
-                float cend[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) cend[c] = s_cend[s * 4 + c];
-                // chunk by chunk; C B^T is released as soon as the last chunk has been read
-#pragma unroll
+                const float ce0 = s_cend[s * 4 + 0], ce1 = s_cend[s * 4 + 1], ce2 = s_cend[s * 4 + 2];
+#pragma unroll 1
                 for (int cc = 0; cc < 2; ++cc) {
-                    // a diagonal first chunk goes second (its partner is all zeros and needs no
-                    // load), so every warp releases C B^T after one load and one chunk's math
-                    const int c = (half == q) ? half + 2 * (1 - cc) : half + 2 * cc;
-                    uint32_t raw[32];
-                    if (c <= q) {
-                        SSD_TMEM_LD32_WAIT(tmem + lane_addr + kColCB + c * 32, raw);
-                    }
-                    if (cc == 1) {
-                        tc_fence_before();
-                        mbar_arrive(bar(BAR_CBFREE));
-                    }
+                    const int c = half + 2 * cc;
+                    uint32_t pk[16];
                     if (c < q) {  // below the diagonal sub-block: factorised decay
-                        const float ce = (c == 0) ? cend[0] : (c == 1) ? cend[1] : cend[2];
+                        uint32_t raw[32];
+                        SSD_TMEM_LD32_WAIT(buf + c * 32, raw);
+                        const float ce = (c == 0) ? ce0 : (c == 1) ? ce1 : ce2;
                         const float uu = dexp<kDecay>(__expf(cs - ce));
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
@@ -684,10 +735,12 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                             const float a1 = __uint_as_float(raw[4 * k + 1]) * uu;
                             const float a2 = __uint_as_float(raw[4 * k + 2]) * uu;
                             const float a3 = __uint_as_float(raw[4 * k + 3]) * uu;
-                            pk[cc][2 * k] = pack_bf16(a0 * v4.x, a1 * v4.y);
-                            pk[cc][2 * k + 1] = pack_bf16(a2 * v4.z, a3 * v4.w);
+                            pk[2 * k] = pack_bf16(a0 * v4.x, a1 * v4.y);
+                            pk[2 * k + 1] = pack_bf16(a2 * v4.z, a3 * v4.w);
                         }
                     } else if (c == q) {  // diagonal sub-block: per-element decay and causal mask
+                        uint32_t raw[32];
+                        SSD_TMEM_LD32_WAIT(buf + c * 32, raw);
 #pragma unroll
                         for (int k = 0; k < 16; ++k) {
                             const int j0 = 2 * k, j1 = 2 * k + 1;  // column within the sub-block
@@ -696,37 +749,30 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                             float v1 = (j1 <= lane) ? __uint_as_float(raw[j1]) * dexp<kDecay>(ex2(csl + m2.y)) : 0.f;
                             if (j0 == lane) v0 += Dh;
                             if (j1 == lane) v1 += Dh;
-                            pk[cc][k] = pack_bf16(v0, v1);
+                            pk[k] = pack_bf16(v0, v1);
                         }
-                    } else {
+                    } else {  // above the diagonal: zeros (the C B^T there is not read)
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) pk[cc][k] = 0u;
+                        for (int k = 0; k < 16; ++k) pk[k] = 0u;
                     }
+                    SSD_TMEM_ST16_WAIT(buf + c * 32, pk);
                 }
-                // the previous block's P X must be done reading P
-                if (u >= 1) live = warp_wait(bar(BAR_G2DONE), (u - 1) & 1, s_abort, prm.status, 12);
-                if (live) {
-                    tc_fence_after();
-                    const int cfirst = (half == q) ? half + 2 : half;
-                    SSD_TMEM_ST16x2_WAIT(tmem + lane_addr + kColP + cfirst * 16, pk[0],
-                                         tmem + lane_addr + kColP + (2 * half + 2 - cfirst) * 16, pk[1]);
-                    tc_fence_before();
-                    mbar_arrive(bar(BAR_SCORES));
-                }
-                // the previous block's output, once P is published (P X of block u-1 is done)
-                if (live && u >= 1) live = store_y(u - 1, ei_prev);
+                tc_fence_before();
+                mbar_arrive(bar(BAR_PREADY + s));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(BAR_ARRFREE + s));  // done with the block's decay terms
+                // the previous block's output
+                if (u >= 1) live = store_y(u - 1, ei_prev);
             }
             ei_prev = ei_cur;
         }
         // output of the last block
-        if (live && nblk > 0) live = warp_wait(bar(BAR_G2DONE), (nblk - 1) & 1, s_abort, prm.status, 18);
         if (live && nblk > 0) live = store_y(nblk - 1, ei_prev);
-    } else if (warp < 18) {
+    } else if (warp < kWarpStore) {
         // ================================================================ state group
-        const int q = warp & 3, half = (warp - 10) >> 2;
-        const int r = q * 32 + lane;  // token row (w o X, y) and state row n (S, H)
+        const int q = warp & 3, half = (warp - kWarpState) >> 2;
+        const int r = q * 32 + lane;  // token row (w o X) and state row n (S, H)
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-        const float Ah = prm.A[hd];
         const int p0 = half * 32;  // this warp's 32 of the 64 p columns
         float Hs[32];              // fp32 running state H[p0 + k][r]
         {
@@ -749,121 +795,143 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
                 *reinterpret_cast<uint4*>(dst + swz(r, half * 4 + c4)) = v4;
             }
         };
+        // H^T of the state entering block 0
         write_sh();
         fence_proxy_async();
-        mbar_arrive(bar(BAR_H));
+        mbar_arrive(bar(BAR_HREADY));
         bool live = __all_sync(0xffffffffu, !*s_abort);
-        bool stopped = false;
-        auto load_dt = [&](int u) {
-            const int tok = tb + u * kBlk + r;
-            if constexpr (kRawDt)
-                return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;
-            else
-                return (u < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;  // used as given
-        };
-        // dt is fetched four blocks ahead: it is a strided gather, and under full HBM load its
-        // latency is microseconds
-        float dt_a = load_dt(0), dt_b = load_dt(1), dt_c = load_dt(2), dt_d = load_dt(3);
-        // raw dt: the head's bias is loaded once, and each block's dt is formed one iteration
-        // before the block needs it, ahead of that iteration's waits (0 past the end)
-        const float dt_bias = (kRawDt && prm.dtm.bias) ? __ldg(prm.dtm.bias + hd) : 0.f;
-        auto form_dt = [&](int u, float v) {
-            const int tok = tb + u * kBlk + r;
-            return (u < nblk && tok < T) ? dt_softplus_clamp(v + dt_bias, prm.dtm) : 0.f;
-        };
-        float dt_next = kRawDt ? form_dt(0, dt_a) : 0.f;
-        float cs_last_prev = 0.f;  // total of the block whose state update is next
-        // iteration k: inputs of block k+1 (w o X), state and output of block k
-        for (int k = -1; k < nblk; ++k) {
-            const int s = (k + 1) & 1;
-            const float dtv = kRawDt ? dt_next : dt_a;  // dt of block k+1
-            dt_a = dt_b;
-            dt_b = dt_c;
-            dt_c = dt_d;
-            dt_d = load_dt(k + 5);
-            if (!live || *s_abort) s_ystop[s] = 1;
-            float cend[4], cs_last;
-            float cs = block_cumsum(dtv * Ah, q, lane, half == 0, s_ytot + s * 4, 3, cs_last, cend);
-            if (kDecay == 2) {
-                cs = dlog<kDecay>(cs);
-                cs_last = dlog<kDecay>(cs_last);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) cend[c] = dlog<kDecay>(cend[c]);
-            }
-            if constexpr (kRawDt) dt_next = form_dt(k + 2, dt_a);  // dt_a now holds block k+2's
-            if (s_ystop[s]) { stopped = true; break; }
-            // ---- w o X of block k+1 (needs S^T(k) accumulated: the MMA has read Xs(k))
-            if (live && k >= 0) live = warp_wait(bar(BAR_ACCS), k & 1, s_abort, prm.status, 13);
-            // ---- publish block k+1's decay arrays for the scores group.  S^T(k) being
-            //      accumulated means the scores group is done with block k-1 (same slot).
-            if (live && k + 1 < nblk) {
-                if (half == 0) {
-                    s_cs[s * kBlk + r] = cs;
-                    s_m[s * kBlk + r] = __log2f(dtv) - cs * kLog2e;   // -inf where dt = 0
-                    // cend[q] (the end of j's 32-token group) and, for lanes 0-3 of quadrant 0,
-                    // cend[lane], by selects: no dynamically indexed local array
-                    const float ce_q = q == 0 ? cend[0] : q == 1 ? cend[1] : q == 2 ? cend[2] : cend[3];
-                    const float ce_l = lane == 0 ? cend[0] : lane == 1 ? cend[1] : lane == 2 ? cend[2] : cend[3];
-                    s_v[s * kBlk + r] = dexp<kDecay>(__expf(ce_q - cs)) * dtv;
-                    if (r < 4) s_cend[s * 4 + r] = ce_l;
-                }
-                mbar_arrive(bar(BAR_PREP0 + s));
-            }
-            if (k >= 0 && live) {
-                // ---- H <- exp(cs_last(k)) H + S(k)
+        float gam = 0.f;  // exp(total log decay) of the block whose S is folded in next
+        // iteration j: fold S of block j into the state; w o X of block j+1; H^T of the state
+        // entering block j+1
+        for (int j = -1; j < nblk && live; ++j) {
+            // ---- S of block j: read it, release the accumulator, H <- exp(cs_last(j)) H + S(j)
+            if (j >= 0) {
+                live = warp_wait(bar(BAR_SDONE), j & 1, s_abort, prm.status, 13);
+                if (!live) break;
                 tc_fence_after();
-                {
-                    uint32_t raw[32];
-                    SSD_TMEM_LD32_WAIT(tmem + lane_addr + kColS + p0, raw);
-                    const float gam = dexp<kDecay>(__expf(cs_last_prev));
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) Hs[j] = fmaf(gam, Hs[j], __uint_as_float(raw[j]));
-                }
+                uint32_t raw[32];
+                SSD_TMEM_LD32_WAIT(tmem + lane_addr + kColS + p0, raw);
                 tc_fence_before();
                 mbar_arrive(bar(BAR_SFREE));
-                // ---- bf16 H_{k+1} for C H^T of block k+1, once C H^T of block k has read H_k
-                live = warp_wait(bar(BAR_YSTDONE), k & 1, s_abort, prm.status, 15);
-                if (live) {
-                    write_sh();
-                    fence_proxy_async();
-                    mbar_arrive(bar(BAR_H));
-                }
-            }
-            // ---- w o X of block k+1 (after the H hand-off: C H^T needs H sooner than the
-            //      state MMA needs w o X)
-            if (live && k + 1 < nblk) {
-                live = warp_wait(bar(BAR_FULLX + (k + 1) % 3), ((k + 1) / 3) & 1, s_abort, prm.status, 14);
-                if (live) {
-                    // w_j x_j as one packed bf16x2 multiply per element pair
-                    const __nv_bfloat162 w2 = __float2bfloat162_rn(dexp<kDecay>(__expf(cs_last - cs)) * dtv);
-                    const uint8_t* src = smem + kXRing + ((k + 1) % 3) * kRegion;
-                    uint8_t* dst = smem + kXs;
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const int c = half * 4 + c4;
-                        uint4 uv = *reinterpret_cast<const uint4*>(src + swz(r, c));
-                        __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&uv);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) e[j] = __hmul2(e[j], w2);
-                        *reinterpret_cast<uint4*>(dst + swz(r, c)) = uv;
-                    }
-                    fence_proxy_async();
-                    mbar_arrive(bar(BAR_XS));
-                }
+                for (int k = 0; k < 32; ++k) Hs[k] = fmaf(gam, Hs[k], __uint_as_float(raw[k]));
             }
-            cs_last_prev = cs_last;
+            // ---- w o X of block j+1 (S of block j has read the previous w o X), with the
+            //      weights w_j = exp(cs_last - cs_j) dt_j the prep warp published
+            if (j + 1 < nblk) {
+                const int s = (j + 1) & 1;
+                live = warp_wait(bar(BAR_PREP + s), ((j + 1) >> 1) & 1, s_abort, prm.status, 16) &&
+                       warp_wait(bar(BAR_FULLX + (j + 1) % 3), ((j + 1) / 3) & 1, s_abort, prm.status, 14);
+                if (!live) break;
+                const __nv_bfloat162 w2 = __float2bfloat162_rn(s_w[s * kBlk + r]);
+                gam = dexp<kDecay>(__expf(s_cslast[s]));
+                const uint8_t* src = smem + kXRing + ((j + 1) % 3) * kRegion;
+                uint8_t* dst = smem + kXs;
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int c = half * 4 + c4;
+                    uint4 uv = *reinterpret_cast<const uint4*>(src + swz(r, c));
+                    __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&uv);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) e[k] = __hmul2(e[k], w2);
+                    *reinterpret_cast<uint4*>(dst + swz(r, c)) = uv;
+                }
+                fence_proxy_async();
+                mbar_arrive(bar(BAR_XSREADY));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(BAR_ARRFREE + s));  // done with the block's decay terms
+            }
+            // ---- bf16 H^T of the state entering block j+1, once C H^T of block j has read
+            //      the previous one
+            if (j >= 0 && j + 1 < nblk) {
+                live = warp_wait(bar(BAR_YSTDONE + (j & 1)), (j >> 1) & 1, s_abort, prm.status, 15);
+                if (!live) break;
+                write_sh();
+                fence_proxy_async();
+                mbar_arrive(bar(BAR_HREADY));
+            }
         }
-        if (!stopped && live && !*s_abort && prm.hf && seg == nseg_u - 1) {
+        if (live && !*s_abort && prm.hf && seg == nseg_u - 1) {
             float* hf = prm.hf + ((size_t)bi * H + hd) * kP * kN;
 #pragma unroll
             for (int j = 0; j < 32; ++j) hf[(size_t)(p0 + j) * kN + r] = Hs[j];
         }
-    } else {
+    } else if (warp == kWarpPrep) {
+        // ================================================================ prep warp
+        // Per-token decay terms of every block, published two blocks ahead of their use: the
+        // prefix sums cs of a = dt*A inside the block (lane l holds tokens l, 32+l, 64+l,
+        // 96+l: four warp scans and the running chunk totals), and from them
+        //   s_cs[i] = cs_i,  s_m[j] = log2(dt_j) - cs_j log2(e),  s_v[j] = exp(cs_e - cs_j) dt_j
+        //   (e = the last token of j's 32-token group),  s_w[j] = exp(cs_last - cs_j) dt_j,
+        //   s_cend = cs at the end of each group,  s_cslast = cs_last.
+        const float Ah = prm.A[hd];
+        const float dt_bias = (kRawDt && prm.dtm.bias) ? __ldg(prm.dtm.bias + hd) : 0.f;
+        auto load4 = [&](int blk, float (&d)[4]) {  // dt as stored, 0 past the end
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int tok = tb + blk * kBlk + 32 * c + lane;
+                d[c] = (blk < nblk && tok < T) ? __ldg(prm.dt + ((size_t)bi * T + tok) * H + hd) : 0.f;
+            }
+        };
+        // dt is fetched three blocks ahead: it is a strided gather, and under full HBM load its
+        // latency is microseconds
+        float da[4], db[4], dc[4];
+        load4(0, da);
+        load4(1, db);
+        load4(2, dc);
+        bool live = __all_sync(0xffffffffu, !*s_abort);
+        for (int blk = 0; blk < nblk && live; ++blk) {
+            const int s = blk & 1;
+            float dtv[4], cs[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int tok = tb + blk * kBlk + 32 * c + lane;
+                dtv[c] = kRawDt ? (tok < T ? dt_softplus_clamp(da[c] + dt_bias, prm.dtm) : 0.f) : da[c];
+                da[c] = db[c];
+                db[c] = dc[c];
+            }
+            load4(blk + 3, dc);
+            // inclusive prefix sums inside each 32-token group, then the running group totals
+#pragma unroll
+            for (int c = 0; c < 4; ++c) cs[c] = dtv[c] * Ah;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float o = __shfl_up_sync(0xffffffffu, cs[c], off);
+                    if (lane >= off) cs[c] += o;
+                }
+            }
+            float cend[4], run = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float tot = __shfl_sync(0xffffffffu, cs[c], 31);
+                cs[c] = dlog<kDecay>(cs[c] + run);
+                run += tot;
+                cend[c] = dlog<kDecay>(run);
+            }
+            const float cs_last = cend[3];
+            // the slot of block blk - 2 must have been read by the scores and state warps
+            if (blk >= 2) live = warp_wait(bar(BAR_ARRFREE + s), ((blk - 2) >> 1) & 1, s_abort, prm.status, 19);
+            if (!live) break;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int j = s * kBlk + 32 * c + lane;
+                s_cs[j] = cs[c];
+                s_m[j] = __log2f(dtv[c]) - cs[c] * kLog2e;  // -inf where dt = 0
+                s_v[j] = dexp<kDecay>(__expf(cend[c] - cs[c])) * dtv[c];
+                s_w[j] = dexp<kDecay>(__expf(cs_last - cs[c])) * dtv[c];
+            }
+            if (lane < 4) s_cend[s * 4 + lane] = lane == 0 ? cend[0] : lane == 1 ? cend[1] : lane == 2 ? cend[2] : cend[3];
+            if (lane == 0) s_cslast[s] = cs_last;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(BAR_PREP + s));
+        }
+    } else if (warp == kWarpStore) {
         // ================================================================ y-store warp
         // One lane writes each block's y tile with a TMA store once the scores group has
         // staged it, waits until the store has read the tile out of shared memory, and
-        // returns the X slot to the producer.  Kept off the scores group's path: a store
-        // queued behind the producer's loads can take microseconds to drain.
+        // returns the X slot to the producer.
         if (lane == 0 && !*s_abort) {
             for (int k = 0; k < nblk; ++k) {
                 const int s3 = k % 3;
@@ -879,7 +947,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     }
 
     // ================================================================ teardown
-    // The MMA lane has seen its final commit land and the producer its last loads; only
+    // Both issuers have seen their final commits land and the producer its last loads; only
     // then is the TMEM released.
     tc_fence_before();
     __syncwarp();
@@ -1007,7 +1075,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
             tc_fence_after();
             const uint32_t slot = sbase + (u % kS) * SP::kSlot;
             const uint64_t dBt = sdesc(slot, kRegion, 1024), dXs = sdesc(slot + kSX, kRegion, 1024);
-#pragma unroll
+#pragma unroll 1
             for (int kk = 0; kk < kBlk / 16; ++kk)
                 mma_ss_w(tmem, dBt + kk * 128, dXs + kk * 128, id_s, (u > 0 || kk > 0) ? 1u : 0u);
             mma_commit_w(bar(SB_EMPTY + u % kS));

@@ -23,8 +23,9 @@ def _dev(d, io):
                 A=f32_tensor(d.A), D=f32_tensor(d.D), w=f32_tensor(d.conv_w), b=f32_tensor(d.conv_b))
 
 
-def _oracle_steps(d, n_steps, act, pairs=None):
-    """Oracle over n_steps; pairs = list of (layer, row) to run (all if None)."""
+def _oracle_steps(d, n_steps, act, pairs=None, mags=False):
+    """Oracle over n_steps; pairs = list of (layer, row) to run (all if None).  With mags,
+    also the term magnitudes of every y and of the final state (fp32 bounds)."""
     if pairs is None:
         pairs = [(l, r) for l in range(d.layers) for r in range(d.b)]
     ls = [p[0] for p in pairs]
@@ -32,11 +33,16 @@ def _oracle_steps(d, n_steps, act, pairs=None):
     # each (layer, row) pair is an independent layer with b = 1
     h = d.h[ls, rs][:, None].astype(np.float64).copy()
     cs = d.conv_state[ls, rs][:, None].astype(np.float64).copy()
-    ys = []
+    hm = np.abs(h)
+    ys, yms = [], []
     for t in range(n_steps):
         s = t % d.ring
-        ys.append(oracle.decode_step(h, cs, d.xbc[s][ls, rs][:, None], d.dt[s][ls, rs][:, None],
-                                     d.A[ls], d.D[ls], d.conv_w[ls], d.conv_b[ls], act=act, G=d.G, N=d.N)[:, 0])
+        args = (d.xbc[s][ls, rs][:, None], d.dt[s][ls, rs][:, None], d.A[ls], d.D[ls], d.conv_w[ls], d.conv_b[ls])
+        if mags:  # before the value step: it reads the window the step starts from
+            yms.append(oracle.decode_step_mag(hm, cs, *args, act=act, G=d.G, N=d.N)[:, 0])
+        ys.append(oracle.decode_step(h, cs, *args, act=act, G=d.G, N=d.N)[:, 0])
+    if mags:
+        return np.stack(ys), h[:, 0], cs[:, 0], np.stack(yms), hm[:, 0]
     return np.stack(ys), h[:, 0], cs[:, 0]
 
 
@@ -49,11 +55,11 @@ def test_decode_steps_vs_oracle(io, act, N, G):
         y = ssd.decode_step(t["h"], t["cs"], t["xbc"][s], t["dt"][s], t["A"], t["D"], t["w"], t["b"], G=G, act=act)
         ys.append(y.float().cpu().numpy())
     torch.cuda.synchronize()
-    y_ref, h_ref, cs_ref = _oracle_steps(d, 6, act)
+    y_ref, h_ref, cs_ref, y_mag, h_mag = _oracle_steps(d, 6, act, mags=True)
     L, B = d.layers, d.b
     y_got = np.stack(ys).reshape(6, L * B, d.H, d.P)
-    check(y_got, y_ref, io, "y")
-    check(t["h"].cpu().numpy().reshape(L * B, d.H, d.P, d.N), h_ref, io, "h")
+    check(y_got, y_ref, io, "y", y_mag)
+    check(t["h"].cpu().numpy().reshape(L * B, d.H, d.P, d.N), h_ref, io, "h", h_mag)
     # the conv window holds raw inputs: exact copies
     np.testing.assert_array_equal(t["cs"].cpu().numpy().reshape(L * B, -1, 3), cs_ref.astype(np.float32))
 

@@ -53,7 +53,7 @@ def test_random_decode_matches_oracle(seed):
             ys.append(y.float().cpu().numpy())
         y_got = np.stack(ys).reshape(c["steps"], L * B, d.H, d.P)
     torch.cuda.synchronize()
-    y_ref, h_ref, cs_ref = _oracle_steps(d, c["steps"], c["act"])
-    check(y_got, y_ref, c["io"], "y %s" % c)
-    check(t["h"].cpu().numpy().reshape(L * B, d.H, d.P, d.N), h_ref, c["io"], "h %s" % c)
+    y_ref, h_ref, cs_ref, y_mag, h_mag = _oracle_steps(d, c["steps"], c["act"], mags=True)
+    check(y_got, y_ref, c["io"], "y %s" % c, y_mag)
+    check(t["h"].cpu().numpy().reshape(L * B, d.H, d.P, d.N), h_ref, c["io"], "h %s" % c, h_mag)
     np.testing.assert_array_equal(t["cs"].cpu().numpy().reshape(L * B, -1, 3), cs_ref.astype(np.float32))

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from ssd_inputs import make_config, make_prefill
-from tests.helpers import check, oracle_subset, prefill_inputs, rel_max, run_prefill
+from tests.helpers import check, oracle_subset, oracle_subset_mag, prefill_inputs, rel_max, run_prefill
 
 pytestmark = pytest.mark.gpu
 
@@ -24,11 +24,19 @@ def _np(t):
     return t.float().cpu().numpy()
 
 
+def _mag(case, nthreads=0):
+    """Term magnitudes for the fp32 per-element bound (None for bf16)."""
+    if case.dtype != "f32":
+        return None, None
+    return oracle_subset_mag(case, range(case.b), range(case.H), nthreads)
+
+
 def _full_check(case, chunk=None, nthreads=0):
     y, hf, _ = run_prefill(ssd, case, chunk)
     y_ref, hf_ref = oracle_subset(case, range(case.b), range(case.H), nthreads)
-    e1 = check(_np(y), y_ref, case.dtype, "y")
-    e2 = check(_np(hf), hf_ref, case.dtype, "h_final")
+    ym, hm = _mag(case, nthreads)
+    e1 = check(_np(y), y_ref, case.dtype, "y", ym)
+    e2 = check(_np(hf), hf_ref, case.dtype, "h_final", hm)
     return e1, e2
 
 
@@ -193,8 +201,9 @@ def test_split_resume(dtype):
     y2, h2 = ssd.prefill(t["x"][:, s:].contiguous(), t["dt"][:, s:].contiguous(), t["A"], t["B"][:, s:].contiguous(),
                          t["C"][:, s:].contiguous(), t["D"], chunk=256, h0=h1)
     torch.cuda.synchronize()
-    check(_np(torch.cat([y1, y2], 1)), _np(y), dtype, "y")
-    check(_np(h2), _np(hf), dtype, "h_final")
+    ym, hm = _mag(case)
+    check(_np(torch.cat([y1, y2], 1)), _np(y), dtype, "y", ym, sides=2)
+    check(_np(h2), _np(hf), dtype, "h_final", hm, sides=2)
 
 
 def test_chunk_length_invariance():
@@ -316,8 +325,11 @@ def test_dt_raw_matches_oracle(dtype, shape, nseg):
     y_ref, hf_ref = oracle.ssd_recurrence(case.x, dt_ref, case.A, case.B, case.C, case.D, case.h0)
     # the kernels form dt in fp32 (softplus within ~2 ulp), the oracle in fp64: rounding
     # the common fp32 metric covers
-    check(_np(y), y_ref, dtype, "y")
-    check(_np(hf), hf_ref, dtype, "h_final")
+    ym = hm = None
+    if dtype == "f32":
+        ym, hm = oracle.ssd_magnitudes(case.x, dt_ref, case.A, case.B, case.C, case.D, case.h0)
+    check(_np(y), y_ref, dtype, "y", ym)
+    check(_np(hf), hf_ref, dtype, "h_final", hm)
 
 
 def test_dt_raw_equals_preprocessed_dt():
