@@ -206,11 +206,26 @@ def test_split_resume(dtype):
     check(_np(h2), _np(hf), dtype, "h_final", hm, sides=2)
 
 
-def test_chunk_length_invariance():
+def test_tensor_core_path_ignores_chunk():
+    """The fused tensor-core kernel (bf16, P = 64, N = 128) evaluates 128-token chunks for
+    every accepted chunk length: the three calls are the same computation, bitwise, and
+    match the oracle."""
     case = make_prefill(1, 1024, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=9)
-    ys = [run_prefill(ssd, case, chunk=L)[0] for L in (64, 128, 256)]
-    for y in ys[:2]:
-        check(_np(y), _np(ys[2]), "bf16", "chunk invariance")
+    runs = [run_prefill(ssd, case, chunk=L)[:2] for L in (64, 128, 256)]
+    for y, hf in runs[:2]:
+        assert torch.equal(y, runs[2][0]) and torch.equal(hf, runs[2][1])
+    y_ref, hf_ref = oracle_subset(case, range(case.b), range(case.H))
+    check(_np(runs[2][0]), y_ref, "bf16", "y")
+    check(_np(runs[2][1]), hf_ref, "bf16", "h_final")
+
+
+@pytest.mark.parametrize("L", [64, 128, 256])
+@pytest.mark.parametrize("dtype,N", [("f32", 64), ("bf16", 64)])
+def test_literal_chunk_length_vs_oracle(dtype, N, L):
+    """The four-kernel path (fp32 inputs, or N = 64) evaluates the chunked form with the
+    chunk length given: every L against the oracle, with a ragged last chunk."""
+    case = make_prefill(1, 3 * L + 37, 4, 64, N, 2, L, dtype, h0_std=0.1, seed=10 + L)
+    _full_check(case, chunk=L)
 
 
 # ------------------------------------------------------------------ edge cases
