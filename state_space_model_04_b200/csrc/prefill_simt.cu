@@ -7,16 +7,24 @@
 // state matrix" property), chunk summary states, a sequential recurrence over them
 // ("Chunked recurrence" property), the state-to-output term and the D skip.
 //
-//   K1 decay_cumsum   cs = inclusive prefix sum of a = dt*A inside each chunk
-//   K2 chunk_state    S_c[p][n] = sum_j exp(cs_last - cs_j) dt_j x_j[p] B_j[n]
-//   K3 state_scan     H_0 = h0, H_{c+1} = exp(cs_last(c)) H_c + S_c  (in place: S -> H_in)
+//   K1 (inside K2)    cs = inclusive prefix sum of a = dt*A inside each chunk
+//   K2 chunk_state    S_c[p][n] = sum_j exp(cs_last - cs_j) dt_j x_j[p] B_j[n], as partial
+//                     sums over slices of the chunk's tokens (one CTA per slice)
+//   K3 state_scan     S_c = the slices' partials summed in order; H_0 = h0,
+//                     H_{c+1} = exp(cs_last(c)) H_c + S_c  (in place: S -> H_in)
 //   K4 chunk_output   y_i = sum_{j<=i} (C_i.B_j) exp(cs_i-cs_j) dt_j x_j
 //                           + exp(cs_i) C_i.H_c + D x_i
+// When (chunks x heads x sequences) alone would leave most SMs idle, the chunk state is
+// split over slices of 32 tokens and the output over 16-row tiles; the partial states are
+// added in a fixed order, so results stay bitwise reproducible.
 //
 // This path serves fp32 inputs: every product and sum is an fp32 FMA (no TF32), and the
 // prefix sums are kept in fp64 (CsT = double) so that exp(cs_i - cs_j) keeps full fp32
 // accuracy even when |cs| reaches several hundred inside a chunk.  A ragged last chunk
 // is handled as if padded with dt = 0 tokens, which leave the state unchanged.
+#include <algorithm>
+#include <cmath>
+
 #include "common.cuh"
 
 namespace ssd {
@@ -30,60 +38,48 @@ constexpr int kP = 64;
 __device__ __forceinline__ float exp_cs(double v) { return (float)exp(v); }
 __device__ __forceinline__ float exp_cs(float v) { return expf(v); }
 
-// ---------------------------------------------------------------- K1
-template <typename CsT>
+// ---------------------------------------------------------------- K1 + K2
+// One CTA per (slice of chunk c, head, sequence).  Every CTA forms its chunk's prefix sums
+// with one block scan (L <= 256 = the CTA's threads); the CTAs of slice 0 store them for K3
+// and K4.  A CTA then accumulates the tokens of its slices -- [32 sl, 32 sl + 32), then
+// every ks-th slice after it -- into its own partial state.
+constexpr int kSliceTokens = 32;
+template <typename IoT, typename CsT, int N>
 __global__ void __launch_bounds__(kThreads)
-decay_cumsum_kernel(int T, int H, int L, int nc, const float* __restrict__ dt, const DtMap dtm,
-                    const float* __restrict__ A, CsT* __restrict__ cs) {
-    const int c = blockIdx.x, hd = blockIdx.y, bi = blockIdx.z;
+chunk_state_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __restrict__ x,
+                   const float* __restrict__ dt, const DtMap dtm, const float* __restrict__ A,
+                   const IoT* __restrict__ Bm, CsT* __restrict__ cs, float* __restrict__ S) {
+    constexpr int KT = kSliceTokens;       // tokens per smem stage
+    constexpr int NT = N / 8;              // thread columns (8 n each)
+    constexpr int PT = kThreads / NT;      // thread rows
+    constexpr int PR = kP / PT;            // p rows per thread
+    const int c = blockIdx.x / ks, sl = blockIdx.x % ks, hd = blockIdx.y, bi = blockIdx.z;
+    const int g = hd / (H / G);
     const int t0 = c * L, Lc = min(L, T - t0);
+
+    __shared__ CsT s_cs[kThreads];
     __shared__ CsT warp_tot[kThreads / 32];
-    __shared__ CsT carry;
-    if (threadIdx.x == 0) carry = CsT(0);
-    __syncthreads();
-    const CsT a_h = (CsT)A[hd];
-    for (int base = 0; base < L; base += kThreads) {
-        const int j = base + threadIdx.x;
-        CsT v = CsT(0);
-        if (j < Lc) v = (CsT)dt_value(dt[((size_t)bi * T + t0 + j) * H + hd], dtm, hd) * a_h;
-        // warp inclusive scan
-        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    __shared__ float sX[KT][kP];
+    __shared__ float sB[KT][N];
+    __shared__ float sW[KT];
+    {
+        // inclusive prefix sum of a = dt*A over the chunk (tokens past its end add 0)
+        const int j = threadIdx.x, lane = j & 31, w = j >> 5;
+        CsT v = j < Lc ? (CsT)dt_value(dt[((size_t)bi * T + t0 + j) * H + hd], dtm, hd) * (CsT)A[hd] : CsT(0);
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            CsT o = __shfl_up_sync(0xffffffffu, v, off);
+            const CsT o = __shfl_up_sync(0xffffffffu, v, off);
             if (lane >= off) v += o;
         }
         if (lane == 31) warp_tot[w] = v;
         __syncthreads();
-        CsT add = carry;
-        for (int k = 0; k < w; ++k) add += warp_tot[k];
-        v += add;
-        if (j < L) cs[(((size_t)bi * H + hd) * nc + c) * L + j] = v;
-        __syncthreads();
-        if (threadIdx.x == kThreads - 1) carry = v;
-        __syncthreads();
+        for (int k = 0; k < w; ++k) v += warp_tot[k];
+        s_cs[j] = v;
+        if (sl == 0 && j < L) cs[(((size_t)bi * H + hd) * nc + c) * L + j] = v;
     }
-}
+    __syncthreads();
+    const CsT cs_last = s_cs[Lc - 1];
 
-// ---------------------------------------------------------------- K2
-template <typename IoT, typename CsT, int N>
-__global__ void __launch_bounds__(kThreads)
-chunk_state_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ x,
-                   const float* __restrict__ dt, const DtMap dtm, const IoT* __restrict__ Bm,
-                   const CsT* __restrict__ cs, float* __restrict__ S) {
-    constexpr int KT = 32;                 // tokens per smem stage
-    constexpr int NT = N / 8;              // thread columns (8 n each)
-    constexpr int PT = kThreads / NT;      // thread rows
-    constexpr int PR = kP / PT;            // p rows per thread
-    const int c = blockIdx.x, hd = blockIdx.y, bi = blockIdx.z;
-    const int g = hd / (H / G);
-    const int t0 = c * L, Lc = min(L, T - t0);
-    const CsT* csc = cs + (((size_t)bi * H + hd) * nc + c) * L;
-    const CsT cs_last = csc[Lc - 1];
-
-    __shared__ float sX[KT][kP];
-    __shared__ float sB[KT][N];
-    __shared__ float sW[KT];
     const int tn = threadIdx.x % NT, tp = threadIdx.x / NT;
     float acc[PR][8];
 #pragma unroll
@@ -91,10 +87,10 @@ chunk_state_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ x
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[i][k] = 0.f;
 
-    for (int k0 = 0; k0 < Lc; k0 += KT) {
+    for (int k0 = sl * KT; k0 < Lc; k0 += ks * KT) {
         if (threadIdx.x < KT) {
             const int t = k0 + threadIdx.x;
-            sW[threadIdx.x] = t < Lc ? exp_cs(cs_last - csc[t]) * dt_value(dt[((size_t)bi * T + t0 + t) * H + hd], dtm, hd) : 0.f;
+            sW[threadIdx.x] = t < Lc ? exp_cs(cs_last - s_cs[t]) * dt_value(dt[((size_t)bi * T + t0 + t) * H + hd], dtm, hd) : 0.f;
         }
         __syncthreads();
         for (int e = threadIdx.x; e < KT * kP; e += kThreads) {
@@ -120,7 +116,7 @@ chunk_state_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ x
         }
         __syncthreads();
     }
-    float* So = S + (((size_t)bi * nc + c) * H + hd) * kP * N;
+    float* So = S + ((((size_t)bi * nc + c) * H + hd) * ks + sl) * kP * N;
 #pragma unroll
     for (int i = 0; i < PR; ++i)
 #pragma unroll
@@ -130,45 +126,53 @@ chunk_state_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ x
 // ---------------------------------------------------------------- K3
 template <typename CsT, int N>
 __global__ void __launch_bounds__(kThreads)
-state_scan_kernel(int T, int H, int L, int nc, const CsT* __restrict__ cs,
+state_scan_kernel(int T, int H, int L, int nc, int ks, const CsT* __restrict__ cs,
                   const float* __restrict__ h0, float* __restrict__ S, float* __restrict__ hf) {
     const int e = blockIdx.x * kThreads + threadIdx.x;  // element of the P x N state
     const int hd = blockIdx.y, bi = blockIdx.z;
     constexpr int PN = kP * N;
     float Hs = h0 ? h0[((size_t)bi * H + hd) * PN + e] : 0.f;
     const CsT* csh = cs + ((size_t)bi * H + hd) * nc * L;
-    const size_t stride = (size_t)H * PN;
-    float* Sp = S + ((size_t)bi * nc * H + hd) * PN + e;
-    float nxt = nc > 0 ? Sp[0] : 0.f;
+    const size_t stride = (size_t)H * ks * PN;          // from one chunk to the next
+    float* Sp = S + ((size_t)bi * nc * H + hd) * ks * PN + e;
+    // S_c: the slices' partial states added in slice order
+    auto chunk_sum = [&](int c) {
+        float v = 0.f;
+        for (int sl = 0; sl < ks; ++sl) v += Sp[(size_t)c * stride + (size_t)sl * PN];
+        return v;
+    };
+    float nxt = nc > 0 ? chunk_sum(0) : 0.f;
     for (int c = 0; c < nc; ++c) {
         const float cur = nxt;
-        if (c + 1 < nc) nxt = Sp[(size_t)(c + 1) * stride];
+        if (c + 1 < nc) nxt = chunk_sum(c + 1);
         const int Lc = min(L, T - c * L);
         const float gam = exp_cs(csh[(size_t)c * L + Lc - 1]);
-        Sp[(size_t)c * stride] = Hs;     // H_in for chunk c
+        Sp[(size_t)c * stride] = Hs;     // H_in for chunk c (slice 0's place)
         Hs = fmaf(gam, Hs, cur);
     }
     if (hf) hf[((size_t)bi * H + hd) * PN + e] = Hs;
 }
 
 // ---------------------------------------------------------------- K4
-// One CTA = 64 output rows of one chunk of one (sequence, head).
-template <typename IoT, typename CsT, int N>
+// One CTA = TR output rows (TR = 16 or 64) of one chunk of one (sequence, head); 16 x 16
+// threads, each RPT = TR / 16 rows x 4 columns (of p for the output, of j for a score tile).
+template <typename IoT, typename CsT, int N, int TR>
 __global__ void __launch_bounds__(kThreads)
-chunk_output_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ x,
+chunk_output_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __restrict__ x,
                     const float* __restrict__ dt, const DtMap dtm, const IoT* __restrict__ Bm,
                     const IoT* __restrict__ Cm, const float* __restrict__ D,
                     const CsT* __restrict__ cs, const float* __restrict__ Hin,
                     IoT* __restrict__ y) {
-    constexpr int TR = 64;          // rows per CTA
+    constexpr int TJ = 64;          // score columns j per tile
+    constexpr int RPT = TR / 16;    // rows per thread
     extern __shared__ float smem[];
     float* sC = smem;               // [TR][N+1]   C rows i
-    float* sK = sC + TR * (N + 1);  // [TR][N+1]   H_in rows p, then B rows j
-    float* sG = sK + TR * (N + 1);  // [TR][TR+1]  masked decayed C.B^T
-    float* sX = sG + TR * (TR + 1); // [TR][kP]    x rows j
+    float* sK = sC + TR * (N + 1);  // [64][N+1]   H_in rows p, then B rows j
+    float* sG = sK + 64 * (N + 1);  // [TR][TJ+1]  masked decayed C.B^T
+    float* sX = sG + TR * (TJ + 1); // [TJ][kP]    x rows j
     __shared__ CsT s_csi[TR];
-    __shared__ CsT s_csj[TR];
-    __shared__ float s_dtj[TR];
+    __shared__ CsT s_csj[TJ];
+    __shared__ float s_dtj[TJ];
 
     const int tiles_per_chunk = (L + TR - 1) / TR;
     const int c = blockIdx.x / tiles_per_chunk, it = blockIdx.x % tiles_per_chunk;
@@ -176,14 +180,14 @@ chunk_output_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ 
     const int t0 = c * L, Lc = min(L, T - t0), i0 = it * TR;
     if (i0 >= Lc) return;
     const CsT* csc = cs + (((size_t)bi * H + hd) * nc + c) * L;
-    const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;  // 16 x 16 threads, 4 x 4 each
+    const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
 
     auto row_ok = [&](int i) { return i < Lc; };
     for (int e = threadIdx.x; e < TR * N; e += kThreads) {
         const int i = e / N, n = e % N;
         sC[i * (N + 1) + n] = row_ok(i0 + i) ? load_io(Cm, (((size_t)bi * T + t0 + i0 + i) * G + g) * N + n) : 0.f;
     }
-    const float* Hc = Hin + (((size_t)bi * nc + c) * H + hd) * kP * N;
+    const float* Hc = Hin + (((size_t)bi * nc + c) * H + hd) * ks * kP * N;
     for (int e = threadIdx.x; e < kP * N; e += kThreads) {
         const int p = e / N, n = e % N;
         sK[p * (N + 1) + n] = Hc[e];
@@ -192,91 +196,91 @@ chunk_output_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ 
     __syncthreads();
 
     // state-to-output term: Y[i][p] = exp(cs_i) * sum_n C[i][n] H[p][n]
-    float acc[4][4];
+    float acc[RPT][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < RPT; ++a)
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[a][q] = 0.f;
     for (int n = 0; n < N; ++n) {
-        float cv[4], hv[4];
+        float cv[RPT], hv[4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) cv[a] = sC[(tr * 4 + a) * (N + 1) + n];
+        for (int a = 0; a < RPT; ++a) cv[a] = sC[(tr * RPT + a) * (N + 1) + n];
 #pragma unroll
         for (int q = 0; q < 4; ++q) hv[q] = sK[(tc * 4 + q) * (N + 1) + n];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < RPT; ++a)
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc[a][q] = fmaf(cv[a], hv[q], acc[a][q]);
     }
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        const float e = exp_cs(s_csi[tr * 4 + a]);
+    for (int a = 0; a < RPT; ++a) {
+        const float e = exp_cs(s_csi[tr * RPT + a]);
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[a][q] *= e;
     }
 
-    // intra-chunk dual form over column tiles j0 <= i0
-    for (int j0 = 0; j0 <= i0; j0 += TR) {
+    // intra-chunk dual form over column tiles j0 <= i0 + TR - 1
+    for (int j0 = 0; j0 < i0 + TR && j0 < Lc; j0 += TJ) {
         __syncthreads();
-        for (int e = threadIdx.x; e < TR * N; e += kThreads) {
+        for (int e = threadIdx.x; e < TJ * N; e += kThreads) {
             const int j = e / N, n = e % N;
             sK[j * (N + 1) + n] = (j0 + j < Lc) ? load_io(Bm, (((size_t)bi * T + t0 + j0 + j) * G + g) * N + n) : 0.f;
         }
-        for (int e = threadIdx.x; e < TR * kP; e += kThreads) {
+        for (int e = threadIdx.x; e < TJ * kP; e += kThreads) {
             const int j = e / kP, p = e % kP;
             sX[j * kP + p] = (j0 + j < Lc) ? load_io(x, (((size_t)bi * T + t0 + j0 + j) * H + hd) * kP + p) : 0.f;
         }
-        if (threadIdx.x < TR) {
+        if (threadIdx.x < TJ) {
             const int j = j0 + threadIdx.x;
             s_csj[threadIdx.x] = j < Lc ? csc[j] : CsT(0);
             s_dtj[threadIdx.x] = j < Lc ? dt_value(dt[((size_t)bi * T + t0 + j) * H + hd], dtm, hd) : 0.f;
         }
         __syncthreads();
-        // G = C_i . B_j over this 64 x 64 tile
-        float gacc[4][4];
+        // G = C_i . B_j over this TR x 64 tile
+        float gacc[RPT][4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < RPT; ++a)
 #pragma unroll
             for (int q = 0; q < 4; ++q) gacc[a][q] = 0.f;
         for (int n = 0; n < N; ++n) {
-            float cv[4], bv[4];
+            float cv[RPT], bv[4];
 #pragma unroll
-            for (int a = 0; a < 4; ++a) cv[a] = sC[(tr * 4 + a) * (N + 1) + n];
+            for (int a = 0; a < RPT; ++a) cv[a] = sC[(tr * RPT + a) * (N + 1) + n];
 #pragma unroll
             for (int q = 0; q < 4; ++q) bv[q] = sK[(tc * 4 + q) * (N + 1) + n];
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < RPT; ++a)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) gacc[a][q] = fmaf(cv[a], bv[q], gacc[a][q]);
         }
         // decay, causal mask and dt_j; the mask is a fixed function of (i, j)
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < RPT; ++a)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const int il = tr * 4 + a, jl = tc * 4 + q;
+                const int il = tr * RPT + a, jl = tc * 4 + q;
                 float v = 0.f;
                 if (j0 + jl <= i0 + il)
                     v = gacc[a][q] * exp_cs(s_csi[il] - s_csj[jl]) * s_dtj[jl];
-                sG[il * (TR + 1) + jl] = v;
+                sG[il * (TJ + 1) + jl] = v;
             }
         __syncthreads();
-        for (int j = 0; j < TR; ++j) {
-            float gv[4], xv[4];
+        for (int j = 0; j < TJ; ++j) {
+            float gv[RPT], xv[4];
 #pragma unroll
-            for (int a = 0; a < 4; ++a) gv[a] = sG[(tr * 4 + a) * (TR + 1) + j];
+            for (int a = 0; a < RPT; ++a) gv[a] = sG[(tr * RPT + a) * (TJ + 1) + j];
 #pragma unroll
             for (int q = 0; q < 4; ++q) xv[q] = sX[j * kP + tc * 4 + q];
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < RPT; ++a)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) acc[a][q] = fmaf(gv[a], xv[q], acc[a][q]);
         }
     }
     const float Dv = D[hd];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        const int i = i0 + tr * 4 + a;
+    for (int a = 0; a < RPT; ++a) {
+        const int i = i0 + tr * RPT + a;
         if (i >= Lc) continue;
         const size_t off = (((size_t)bi * T + t0 + i) * H + hd) * kP;
 #pragma unroll
@@ -287,37 +291,66 @@ chunk_output_kernel(int T, int H, int G, int L, int nc, const IoT* __restrict__ 
     }
 }
 
+int sm_count_simt() {
+    static int n = 0;
+    if (n <= 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+// Slices per chunk for the chunk-state pass: enough CTAs for two per SM when (chunks x
+// heads x sequences) alone fall short, at most one per 32 tokens of the chunk, and at most
+// 256 MB of partial states.
+int state_slices(int b, int T, int H, int N, int L) {
+    const int nc = (T + L - 1) / L;
+    const double units = (double)nc * H * b;
+    int ks = (int)std::ceil(2.0 * sm_count_simt() / std::max(units, 1.0));
+    ks = std::max(1, std::min(ks, L / kSliceTokens));
+    while (ks > 1 && units * ks * kP * N * sizeof(float) > 256.0 * 1024 * 1024) --ks;
+    return ks;
+}
+
+template <typename IoT, typename CsT, int N, int TR>
+int launch_output(int b, int T, int H, int G, int L, int nc, int ks, const IoT* x, const float* dt, const DtMap& dtm,
+                  const IoT* Bm, const IoT* Cm, const float* D, const CsT* cs, const float* S, void* y, cudaStream_t s) {
+    const size_t smem = sizeof(float) * (TR * (N + 1) + 64 * (N + 1) + TR * 65 + 64 * kP);
+    auto k4 = chunk_output_kernel<IoT, CsT, N, TR>;
+    if (const int st = smem_limit_once((const void*)k4, (int)smem)) return st;
+    LaunchScope ls("simt_chunk_output", s);
+    k4<<<dim3(nc * ((L + TR - 1) / TR), H, b), kThreads, smem, s>>>(T, H, G, L, nc, ks, x, dt, dtm, Bm, Cm, D, cs, S,
+                                                                     static_cast<IoT*>(y));
+    return SSD_OK;
+}
+
 template <typename IoT, typename CsT, int N>
 int run(int b, int T, int H, int G, int L, const void* x, const float* dt, const DtMap dtm, const float* A,
         const void* Bm, const void* Cm, const float* D, const float* h0, void* y, float* hf,
         char* ws, cudaStream_t s) {
     const int nc = (T + L - 1) / L;
+    const int ks = state_slices(b, T, H, N, L);
     CsT* cs = reinterpret_cast<CsT*>(ws);
     float* S = reinterpret_cast<float*>(ws + round_up((size_t)b * H * nc * L * sizeof(CsT), 256));
     const IoT* xi = static_cast<const IoT*>(x);
     const IoT* Bi = static_cast<const IoT*>(Bm);
     const IoT* Ci = static_cast<const IoT*>(Cm);
-    dim3 gchunk(nc, H, b);
-    {
-        LaunchScope ls("simt_decay_cumsum", s);
-        decay_cumsum_kernel<CsT><<<gchunk, kThreads, 0, s>>>(T, H, L, nc, dt, dtm, A, cs);
-    }
     {
         LaunchScope ls("simt_chunk_state", s);
-        chunk_state_kernel<IoT, CsT, N><<<gchunk, kThreads, 0, s>>>(T, H, G, L, nc, xi, dt, dtm, Bi, cs, S);
+        chunk_state_kernel<IoT, CsT, N><<<dim3(nc * ks, H, b), kThreads, 0, s>>>(T, H, G, L, nc, ks, xi, dt, dtm, A, Bi,
+                                                                                  cs, S);
     }
     {
         LaunchScope ls("simt_state_scan", s);
-        state_scan_kernel<CsT, N><<<dim3(kP * N / kThreads, H, b), kThreads, 0, s>>>(T, H, L, nc, cs, h0, S, hf);
+        state_scan_kernel<CsT, N><<<dim3(kP * N / kThreads, H, b), kThreads, 0, s>>>(T, H, L, nc, ks, cs, h0, S, hf);
     }
-    const size_t smem = sizeof(float) * (2 * 64 * (N + 1) + 64 * 65 + 64 * kP);
-    auto k4 = chunk_output_kernel<IoT, CsT, N>;
-    if (const int st = smem_limit_once((const void*)k4, (int)smem)) return st;
-    {
-        LaunchScope ls("simt_chunk_output", s);
-        k4<<<dim3(nc * ((L + 63) / 64), H, b), kThreads, smem, s>>>(T, H, G, L, nc, xi, dt, dtm, Bi, Ci, D, cs, S,
-                                                                     static_cast<IoT*>(y));
-    }
+    // 16-row output tiles when 64-row tiles would not give every SM two CTAs
+    const bool small = (double)nc * ((L + 63) / 64) * H * b < 2.0 * sm_count_simt();
+    const int st = small ? launch_output<IoT, CsT, N, 16>(b, T, H, G, L, nc, ks, xi, dt, dtm, Bi, Ci, D, cs, S, y, s)
+                         : launch_output<IoT, CsT, N, 64>(b, T, H, G, L, nc, ks, xi, dt, dtm, Bi, Ci, D, cs, S, y, s);
+    if (st != SSD_OK) return st;
     SSD_CUDA_TRY(cudaGetLastError());
     return SSD_OK;
 }
@@ -328,7 +361,7 @@ size_t prefill_simt_workspace_bytes(int b, int T, int H, int N, int L, int io) {
     const int nc = (T + L - 1) / L;
     const size_t cs_elem = io == SSD_F32 ? sizeof(double) : sizeof(float);
     return round_up((size_t)b * H * nc * L * cs_elem, 256) +
-           round_up((size_t)b * nc * H * kP * N * sizeof(float), 256);
+           round_up((size_t)b * nc * H * state_slices(b, T, H, N, L) * kP * N * sizeof(float), 256);
 }
 
 int launch_prefill_simt(int b, int T, int H, int N, int G, int L, int io, const void* x,
