@@ -38,6 +38,22 @@ constexpr int kP = 64;
 __device__ __forceinline__ float exp_cs(double v) { return (float)exp(v); }
 __device__ __forceinline__ float exp_cs(float v) { return expf(v); }
 
+// Runs `count` (a multiple of the block size) element copies through registers, eight per
+// thread at a time: the group's global loads are all in flight before its stores.
+template <int kCount, typename Load, typename Store>
+__device__ __forceinline__ void copy_grouped(Load load, Store store) {
+    constexpr int kPer = kCount / kThreads, kGrp = kPer < 8 ? kPer : 8;
+    static_assert(kCount % kThreads == 0 && kPer % kGrp == 0, "tile size");
+#pragma unroll 1
+    for (int k0 = 0; k0 < kPer; k0 += kGrp) {
+        float r[kGrp];
+#pragma unroll
+        for (int k = 0; k < kGrp; ++k) r[k] = load(threadIdx.x + (k0 + k) * kThreads);
+#pragma unroll
+        for (int k = 0; k < kGrp; ++k) store(threadIdx.x + (k0 + k) * kThreads, r[k]);
+    }
+}
+
 // ---------------------------------------------------------------- K1 + K2
 // One CTA per (slice of chunk c, head, sequence).  Every CTA forms its chunk's prefix sums
 // with one block scan (L <= 256 = the CTA's threads); the CTAs of slice 0 store them for K3
@@ -93,14 +109,18 @@ chunk_state_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __rest
             sW[threadIdx.x] = t < Lc ? exp_cs(cs_last - s_cs[t]) * dt_value(dt[((size_t)bi * T + t0 + t) * H + hd], dtm, hd) : 0.f;
         }
         __syncthreads();
-        for (int e = threadIdx.x; e < KT * kP; e += kThreads) {
-            const int j = e / kP, p = e % kP, t = k0 + j;
-            sX[j][p] = t < Lc ? sW[j] * load_io(x, (((size_t)bi * T + t0 + t) * H + hd) * kP + p) : 0.f;
-        }
-        for (int e = threadIdx.x; e < KT * N; e += kThreads) {
-            const int j = e / N, n = e % N, t = k0 + j;
-            sB[j][n] = t < Lc ? load_io(Bm, (((size_t)bi * T + t0 + t) * G + g) * N + n) : 0.f;
-        }
+        copy_grouped<KT * kP>(
+            [&](int e) {
+                const int t = k0 + e / kP;
+                return t < Lc ? load_io(x, (((size_t)bi * T + t0 + t) * H + hd) * kP + e % kP) : 0.f;
+            },
+            [&](int e, float v) { sX[e / kP][e % kP] = sW[e / kP] * v; });
+        copy_grouped<KT * N>(
+            [&](int e) {
+                const int t = k0 + e / N;
+                return t < Lc ? load_io(Bm, (((size_t)bi * T + t0 + t) * G + g) * N + e % N) : 0.f;
+            },
+            [&](int e, float v) { sB[e / N][e % N] = v; });
         __syncthreads();
 #pragma unroll 4
         for (int j = 0; j < KT; ++j) {
@@ -183,15 +203,14 @@ chunk_output_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __res
     const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
 
     auto row_ok = [&](int i) { return i < Lc; };
-    for (int e = threadIdx.x; e < TR * N; e += kThreads) {
-        const int i = e / N, n = e % N;
-        sC[i * (N + 1) + n] = row_ok(i0 + i) ? load_io(Cm, (((size_t)bi * T + t0 + i0 + i) * G + g) * N + n) : 0.f;
-    }
     const float* Hc = Hin + (((size_t)bi * nc + c) * H + hd) * ks * kP * N;
-    for (int e = threadIdx.x; e < kP * N; e += kThreads) {
-        const int p = e / N, n = e % N;
-        sK[p * (N + 1) + n] = Hc[e];
-    }
+    copy_grouped<TR * N>(
+        [&](int e) {
+            const int i = e / N;
+            return row_ok(i0 + i) ? load_io(Cm, (((size_t)bi * T + t0 + i0 + i) * G + g) * N + e % N) : 0.f;
+        },
+        [&](int e, float v) { sC[(e / N) * (N + 1) + e % N] = v; });
+    copy_grouped<kP * N>([&](int e) { return Hc[e]; }, [&](int e, float v) { sK[(e / N) * (N + 1) + e % N] = v; });
     if (threadIdx.x < TR) s_csi[threadIdx.x] = row_ok(i0 + threadIdx.x) ? csc[i0 + threadIdx.x] : CsT(0);
     __syncthreads();
 
@@ -222,14 +241,18 @@ chunk_output_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __res
     // intra-chunk dual form over column tiles j0 <= i0 + TR - 1
     for (int j0 = 0; j0 < i0 + TR && j0 < Lc; j0 += TJ) {
         __syncthreads();
-        for (int e = threadIdx.x; e < TJ * N; e += kThreads) {
-            const int j = e / N, n = e % N;
-            sK[j * (N + 1) + n] = (j0 + j < Lc) ? load_io(Bm, (((size_t)bi * T + t0 + j0 + j) * G + g) * N + n) : 0.f;
-        }
-        for (int e = threadIdx.x; e < TJ * kP; e += kThreads) {
-            const int j = e / kP, p = e % kP;
-            sX[j * kP + p] = (j0 + j < Lc) ? load_io(x, (((size_t)bi * T + t0 + j0 + j) * H + hd) * kP + p) : 0.f;
-        }
+        copy_grouped<TJ * N>(
+            [&](int e) {
+                const int j = e / N;
+                return (j0 + j < Lc) ? load_io(Bm, (((size_t)bi * T + t0 + j0 + j) * G + g) * N + e % N) : 0.f;
+            },
+            [&](int e, float v) { sK[(e / N) * (N + 1) + e % N] = v; });
+        copy_grouped<TJ * kP>(
+            [&](int e) {
+                const int j = e / kP;
+                return (j0 + j < Lc) ? load_io(x, (((size_t)bi * T + t0 + j0 + j) * H + hd) * kP + e % kP) : 0.f;
+            },
+            [&](int e, float v) { sX[e] = v; });
         if (threadIdx.x < TJ) {
             const int j = j0 + threadIdx.x;
             s_csj[threadIdx.x] = j < Lc ? csc[j] : CsT(0);
