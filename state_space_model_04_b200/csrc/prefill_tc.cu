@@ -144,6 +144,9 @@ struct TcParams {
     const float* A;
     const float* D;
     const float* h0;
+    const float* h0_split;       // h0 as read by the first segment of a split unit: h0 itself, or
+                                 // a copy when h0 and hf are one buffer (the unit's last segment
+                                 // writes hf while its first may not have started)
     float* hf;
     __nv_bfloat16* y;
     int* status;
@@ -153,9 +156,12 @@ struct TcParams {
     // tseg tokens (a multiple of kBlk; the last may be shorter).  The fused kernel's CTAs
     // walk n_full whole units, then the split units' segments in order.
     int n_full, tseg, nseg;
-    float* seg_state;            // [su][nseg-1][P][N] fp32: a segment's local end state, then
-                                 // (after the scan) the state entering the next segment
+    float* seg_state;            // [su][nseg-1][P][N] fp32: the end state of segment q started
+                                 // from zero, except segment 0, which starts from h0; with
+                                 // seg_prefix, the prefix pass has turned each into the state
+                                 // entering segment q + 1
     float* seg_logdecay;         // [su][nseg-1]: sum of dt*A over a segment
+    int seg_prefix;
     unsigned long long wait_ns;  // limit of every bounded wait
     int starve;                  // failure-detection test: the producer issues no loads
 };
@@ -205,6 +211,19 @@ __device__ __forceinline__ bool mbar_try_sleep(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Programmatic dependent launch.  A grid launched with programmatic stream serialization
+// may start while the grid before it in the stream is still running: griddep_wait() blocks
+// until that grid has completed and its writes are visible, and griddep_launch() lets the
+// next grid in the stream start before this one ends.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Records a failure in the status word (the first one wins).  The word is cleared by the
+// grid that runs ahead of every prefill, so the write waits until that grid is done.
+__device__ __noinline__ void report_status(int* status, int code) {
+    griddep_wait();
+    atomicCAS(status, 0, code);
+}
+
 // Bounded wait for the phase with `parity` to complete.  Returns false (and makes every
 // other role give up) if the CTA is aborting or the limit expires.  The first test is
 // inline; the waiting loop is one out-of-line copy shared by every call site, which keeps
@@ -217,7 +236,7 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
         if (*abort_flag) return false;
         if (globaltimer() - t0 > s_wait_ns) {
             *abort_flag = 1;
-            atomicCAS(status, 0, SSD_ERR_TIMEOUT | (where << 8));
+            report_status(status, SSD_ERR_TIMEOUT | (where << 8));
             return false;
         }
     }
@@ -516,7 +535,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 
     if (threadIdx.x == 0) {
         const bool misaligned = (sbase & 1023u) != 0;  // swizzled layouts need a 1024-byte base
-        if (misaligned) atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (1 << 8));
+        if (misaligned) report_status(prm.status, SSD_ERR_INTERNAL | (1 << 8));
         for (int i = 0; i < BAR_COUNT; ++i) mbar_init(bar(i), bar_count(i));
         *s_abort = misaligned ? 1 : 0;
         s_wait_ns = prm.wait_ns;
@@ -525,7 +544,7 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
     const uint32_t tmem = tmem_alloc_cta(s_tmem, kTmemCols, warp == 1);  // warp 1 owns the TMEM
     if (tmem == kTmemSentinel) {
         *s_abort = 1;
-        atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (3 << 8));
+        report_status(prm.status, SSD_ERR_INTERNAL | (3 << 8));
     }
 
     if (warp == 0) {
@@ -775,13 +794,32 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
         const int p0 = half * 32;  // this warp's 32 of the 64 p columns
         float Hs[32];              // fp32 running state H[p0 + k][r]
-        {
-            // state entering the segment: h0 for the first, the scanned segment states after it
-            const float* h0 = seg > 0 ? prm.seg_state + ((size_t)(u - prm.n_full) * (prm.nseg - 1) + seg - 1) * kP * kN
-                              : prm.h0 ? prm.h0 + (size_t)u * kP * kN
-                                       : nullptr;
+        if (seg == 0) {
+            // state entering a whole unit or a first segment: h0
+            const float* h0 = u < prm.n_full ? prm.h0 : prm.h0_split;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) Hs[k] = h0 ? h0[(size_t)(p0 + k) * kN + r] : 0.f;
+            for (int k = 0; k < 32; ++k) Hs[k] = h0 ? h0[(size_t)u * kP * kN + (size_t)(p0 + k) * kN + r] : 0.f;
+        } else {
+            // state entering segment seg: the end states of the segments before it, folded in
+            // order, H <- exp(logdecay_q) H + H_q (already folded by the prefix pass when a
+            // sequence has many segments).  This grid may start before the grid that wrote
+            // them has ended.
+            griddep_wait();
+            const size_t o = (size_t)(u - prm.n_full) * (prm.nseg - 1);
+            const float* st = prm.seg_state + o * kP * kN + r;
+            const int first = prm.seg_prefix ? seg - 1 : 0;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) Hs[k] = st[(size_t)first * kP * kN + (size_t)(p0 + k) * kN];
+#pragma unroll 1
+            for (int q = first + 1; q < seg; ++q) {
+                const float gq = __expf(prm.seg_logdecay[o + q]);
+                const float* sq = st + (size_t)q * kP * kN;
+                float v[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) v[k] = sq[(size_t)(p0 + k) * kN];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) Hs[k] = fmaf(gq, Hs[k], v[k]);
+            }
         }
         auto write_sh = [&]() {  // bf16 H^T row r, chunks [4 half, 4 half + 4)
             uint8_t* dst = smem + kSH;
@@ -948,7 +986,8 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 
     // ================================================================ teardown
     // Both issuers have seen their final commits land and the producer its last loads; only
-    // then is the TMEM released.
+    // then is the TMEM released.  The grid ends after the one before it in the stream.
+    griddep_wait();
     tc_fence_before();
     __syncwarp();
     __syncthreads();
@@ -1027,7 +1066,7 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
 
     if (threadIdx.x == 0) {
         const bool misaligned = (sbase & 1023u) != 0;
-        if (misaligned) atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (2 << 8));
+        if (misaligned) report_status(prm.status, SSD_ERR_INTERNAL | (2 << 8));
         for (int i = 0; i < SB_COUNT; ++i) mbar_init(bar(i), (i >= SB_XS && i < SB_XS + 3) ? kGroupThreads : 1);
         *s_abort = misaligned ? 1 : 0;
         s_wait_ns = prm.wait_ns;
@@ -1037,8 +1076,11 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
     const uint32_t tmem = tmem_alloc_cta(s_tmem, SP::kTmemCols, warp == 1);  // warp 1 owns the TMEM
     if (tmem == kTmemSentinel) {
         *s_abort = 1;
-        atomicCAS(prm.status, 0, SSD_ERR_INTERNAL | (4 << 8));
+        report_status(prm.status, SSD_ERR_INTERNAL | (4 << 8));
     }
+    // the fused pass may be scheduled now: only its segments after the first read what this
+    // grid writes, and they wait for it to end
+    griddep_launch();
     constexpr int kS = SP::kSlots;
 
     if (warp == 0) {
@@ -1162,13 +1204,25 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
             if (!*s_abort) {
                 const size_t o = (size_t)(su0 + h) * (prm.nseg - 1) + seg;
                 float* dst = prm.seg_state + o * kP * kN;
+                if (seg == 0 && prm.h0) {
+                    // the first segment's end state starts from h0: exp(logdecay) h0 + H_loc
+                    const float gam = __expf(later);
+                    const float* h0 = prm.h0 + (size_t)(u0 + h) * kP * kN;
 #pragma unroll
-                for (int j = 0; j < kCols; ++j) dst[(size_t)(pbase + j) * kN + r] = __uint_as_float(raw[j]);
+                    for (int j = 0; j < kCols; ++j) {
+                        const size_t e = (size_t)(pbase + j) * kN + r;
+                        dst[e] = fmaf(gam, h0[e], __uint_as_float(raw[j]));
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < kCols; ++j) dst[(size_t)(pbase + j) * kN + r] = __uint_as_float(raw[j]);
+                }
                 if (r == 0 && (kHP == 2 || half == 0)) prm.seg_logdecay[o] = later;
             }
         }
     }
 
+    griddep_wait();  // the grid ends after the one before it in the stream
     tc_fence_before();
     __syncwarp();
     __syncthreads();
@@ -1181,6 +1235,40 @@ ssd_segment_state_kernel(const __grid_constant__ TcParams prm) {
 
 int sm_count();
 
+// Clears the status word ahead of a prefill and lets the prefill's first grid start at once
+// (that grid's writes to the word wait for this one).
+__global__ void ssd_status_reset_kernel(int* status) {
+    if (threadIdx.x == 0) *status = 0;
+    griddep_launch();
+}
+
+// Launches `k` with programmatic stream serialization: it may start while the grid ahead of
+// it in the stream still runs, and waits (griddep_wait) where it needs that grid's results.
+template <typename Param>
+cudaError_t launch_pdl(void (*k)(Param), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                       const Param& prm) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, prm);
+}
+
+int reset_status(int* status, cudaStream_t s) {
+    {
+        LaunchScope ls("ssd_status_reset", s);
+        ssd_status_reset_kernel<<<1, 32, 0, s>>>(status);
+    }
+    SSD_CUDA_TRY(cudaGetLastError());
+    return SSD_OK;
+}
+
 // Launches the state pass over the split units [n_full, n_full + n_split): two heads per CTA
 // where both heads of every pair share a B/C group, one otherwise.
 template <int kHP>
@@ -1191,9 +1279,8 @@ int launch_state_pass_hp(const TcParams& prm, int decay, unsigned grid, cudaStre
     if (const int st = smem_limit_once((const void*)k, (int)SPass<kHP>::kSmem)) return st;
     {
         LaunchScope ls("ssd_segment_state", s);
-        k<<<grid, kSThreads, SPass<kHP>::kSmem, s>>>(prm);
+        SSD_CUDA_TRY(launch_pdl(k, grid, kSThreads, SPass<kHP>::kSmem, s, prm));
     }
-    SSD_CUDA_TRY(cudaGetLastError());
     return SSD_OK;
 }
 int launch_state_pass(const TcParams& prm, int n_split, int decay, cudaStream_t s) {
@@ -1207,39 +1294,40 @@ int launch_state_pass(const TcParams& prm, int n_split, int decay, cudaStream_t 
     return pair ? launch_state_pass_hp<2>(prm, decay, grid, s) : launch_state_pass_hp<1>(prm, decay, grid, s);
 }
 
-// Entering state of every segment after the first, in place of the local states:
-// H_in(s + 1) = exp(logdecay(s)) H_in(s) + H_loc(s), H_in(0) = h0.  Each (sequence,
-// head) state is spread over kScanSplit CTAs; a thread carries kScanPer entries through
-// the segments, loading kScanBatch segments' worth before the dependent updates.
+// Folding kernel geometry: each (sequence, head) state is spread over kScanSplit CTAs; a
+// thread carries kScanPer entries through the stretches, loading kScanBatch stretches'
+// worth before the dependent updates.
 constexpr int kScanSplit = 8, kScanThreads = 128, kScanPer = kP * kN / (kScanSplit * kScanThreads), kScanBatch = 4;
-__global__ void __launch_bounds__(kScanThreads) ssd_segment_scan_kernel(const float* h0, float* seg_state,
-                                                                         const float* seg_logdecay, int n_full,
-                                                                         int nseg) {
-    const int su = blockIdx.x;  // split unit
-    const size_t o = (size_t)su * (nseg - 1);
-    const int e0 = blockIdx.z * (kP * kN / kScanSplit) + threadIdx.x;  // entries e0 + kScanThreads * k
-    const float* h0p = h0 ? h0 + (size_t)(n_full + su) * kP * kN : nullptr;
+
+// Prefix pass over a split unit's segment end states, in place: H_q <- exp(logdecay_q)
+// H_{q-1} + H_q for q = 1 .. nseg - 2, so that H_q becomes the state entering segment q + 1
+// (H_0 already starts from h0).  Used when a sequence has more segments than the fused
+// kernel folds itself; the same operations in the same order as that fold.
+__global__ void __launch_bounds__(kScanThreads) ssd_segment_prefix_kernel(float* seg_state, const float* seg_logdecay,
+                                                                           int nseg) {
+    griddep_launch();  // the fused pass may be scheduled; its later segments wait for this grid
+    griddep_wait();    // the state pass's end states
+    const size_t o = (size_t)blockIdx.x * (nseg - 1);
+    float* st = seg_state + o * kP * kN + blockIdx.z * (kP * kN / kScanSplit) + threadIdx.x;
     float run[kScanPer];
 #pragma unroll
-    for (int k = 0; k < kScanPer; ++k) run[k] = h0p ? h0p[e0 + kScanThreads * k] : 0.f;
-    for (int s0 = 0; s0 + 1 < nseg; s0 += kScanBatch) {
+    for (int k = 0; k < kScanPer; ++k) run[k] = st[kScanThreads * k];
+    for (int q0 = 1; q0 + 1 < nseg; q0 += kScanBatch) {
         float v[kScanBatch][kScanPer], gam[kScanBatch];
 #pragma unroll
         for (int j = 0; j < kScanBatch; ++j) {
-            const bool in = s0 + j + 1 < nseg;
-            gam[j] = in ? __expf(seg_logdecay[o + s0 + j]) : 0.f;
-            const float* w = seg_state + (o + s0 + j) * kP * kN;
+            const bool in = q0 + j + 1 < nseg;
+            gam[j] = in ? __expf(seg_logdecay[o + q0 + j]) : 0.f;
 #pragma unroll
-            for (int k = 0; k < kScanPer; ++k) v[j][k] = in ? w[e0 + kScanThreads * k] : 0.f;
+            for (int k = 0; k < kScanPer; ++k) v[j][k] = in ? st[(size_t)(q0 + j) * kP * kN + kScanThreads * k] : 0.f;
         }
 #pragma unroll
         for (int j = 0; j < kScanBatch; ++j) {
-            if (s0 + j + 1 >= nseg) break;
-            float* w = seg_state + (o + s0 + j) * kP * kN;
+            if (q0 + j + 1 >= nseg) break;
 #pragma unroll
             for (int k = 0; k < kScanPer; ++k) {
                 run[k] = fmaf(gam[j], run[k], v[j][k]);
-                w[e0 + kScanThreads * k] = run[k];
+                st[(size_t)(q0 + j) * kP * kN + kScanThreads * k] = run[k];
             }
         }
     }
@@ -1349,6 +1437,7 @@ constexpr double kStatePassPerBlock = 0.7;  // single-head state pass; the paire
 constexpr double kCtaStartBlocks = 2.0;
 constexpr double kScanPerSegment = 0.4;
 constexpr double kSplitFixedBlocks = 5.0;
+constexpr int kFoldMax = 5;  // the fused kernel folds up to this many segment states itself
 std::atomic<int> g_force_nseg{0};     // 0: cost model
 std::atomic<int> g_force_nfull{-1};   // -1: every unit split when nseg > 1
 std::atomic<int> g_decay_mode{0};
@@ -1401,11 +1490,25 @@ SplitPlan plan_split(int b, int T, int H) {
 
 int prefill_tc_segments(int b, int T, int H) { return plan_split(b, T, H).nseg; }
 
+// Workspace: the status word, then (split sequences only) the segments' end states, their
+// log decays, and room for a copy of the split units' h0.
+struct SplitLayout {
+    size_t state, logdecay, h0copy, bytes;
+};
+SplitLayout split_layout(int b, int H, const SplitPlan& sp) {
+    const size_t n_split = (size_t)(b * H - sp.n_full), units = n_split * (sp.nseg - 1);
+    SplitLayout l;
+    l.state = kSegOffset;
+    l.logdecay = l.state + align256(units * kP * kN * sizeof(float));
+    l.h0copy = l.logdecay + align256(units * sizeof(float));
+    l.bytes = l.h0copy + align256(n_split * kP * kN * sizeof(float));
+    return l;
+}
+
 size_t prefill_tc_workspace_bytes(int b, int T, int H) {
     const SplitPlan sp = plan_split(b, T, H);
     if (sp.nseg == 1) return kSegOffset;
-    const size_t units = (size_t)(b * H - sp.n_full) * (sp.nseg - 1);
-    return kSegOffset + align256(units * kP * kN * sizeof(float)) + align256(units * sizeof(float));
+    return split_layout(b, H, sp).bytes;
 }
 
 namespace {
@@ -1456,30 +1559,51 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     prm.nseg = sp.nseg;
     prm.tseg = sp.tseg;
     const int n_split = b * H - sp.n_full;
-    const size_t units = (size_t)n_split * (prm.nseg - 1);
-    prm.seg_state = reinterpret_cast<float*>(static_cast<char*>(ws) + kSegOffset);
-    prm.seg_logdecay = reinterpret_cast<float*>(static_cast<char*>(ws) + kSegOffset +
-                                                align256(units * kP * kN * sizeof(float)));
+    prm.h0_split = h0;
+    if (prm.nseg > 1) {
+        const SplitLayout l = split_layout(b, H, sp);
+        char* w = static_cast<char*>(ws);
+        prm.seg_state = reinterpret_cast<float*>(w + l.state);
+        prm.seg_logdecay = reinterpret_cast<float*>(w + l.logdecay);
+        if (h0 && h0 == hf) {
+            // the first segment of a split unit reads h0 from a copy: the unit's last segment
+            // overwrites h0 with h_final, and nothing orders the two CTAs
+            float* cp = reinterpret_cast<float*>(w + l.h0copy);
+            const size_t off = (size_t)sp.n_full * kP * kN;
+            SSD_CUDA_TRY(cudaMemcpyAsync(cp + off, h0 + off, (size_t)n_split * kP * kN * sizeof(float),
+                                         cudaMemcpyDeviceToDevice, s));
+            prm.h0_split = cp;
+        }
+    }
     const unsigned long long starve_ns = g_starve_ns.exchange(0);
     prm.starve = starve_ns != 0;
     prm.wait_ns = starve_ns ? starve_ns : kWaitLimitNs;
-    SSD_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), s));
-    if (prm.nseg > 1) {
-        // local end states of all segments but the last, then their scan
-        if ((st = launch_state_pass(prm, n_split, decay, s)) != SSD_OK) return st;
-        {
-            LaunchScope ls("ssd_segment_scan", s);
-            ssd_segment_scan_kernel<<<dim3(n_split, 1, kScanSplit), kScanThreads, 0, s>>>(
-                h0, prm.seg_state, prm.seg_logdecay, prm.n_full, prm.nseg);
-        }
-        SSD_CUDA_TRY(cudaGetLastError());
+    // Grids in a row, each allowed to start before the one ahead ends: the status reset; for
+    // split sequences the end states of all segments but the last, and when there are many
+    // segments their prefix pass; the fused pass, whose later segments fold in the end states
+    // (or read the prefix) once the grid before has ended
+    prm.seg_prefix = prm.nseg - 1 > kFoldMax;
+    if ((st = reset_status(prm.status, s)) != SSD_OK) return st;
+    if (prm.nseg > 1 && (st = launch_state_pass(prm, n_split, decay, s)) != SSD_OK) return st;
+    if (prm.seg_prefix) {
+        LaunchScope ls("ssd_segment_prefix", s);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)n_split, 1, kScanSplit);
+        cfg.blockDim = dim3(kScanThreads);
+        cfg.stream = s;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        SSD_CUDA_TRY(cudaLaunchKernelEx(&cfg, ssd_segment_prefix_kernel, prm.seg_state,
+                                        (const float*)prm.seg_logdecay, prm.nseg));
     }
     if ((st = smem_limit_once((const void*)fused, (int)kSmemBytes)) != SSD_OK) return st;
     {
         LaunchScope ls("ssd_prefill_fused", s);
-        fused<<<(unsigned)(prm.n_full + (size_t)n_split * prm.nseg), kThreads, kSmemBytes, s>>>(prm);
+        SSD_CUDA_TRY(launch_pdl(fused, (unsigned)(prm.n_full + (size_t)n_split * prm.nseg), kThreads, kSmemBytes, s, prm));
     }
-    SSD_CUDA_TRY(cudaGetLastError());
     return SSD_OK;
 }
 
@@ -1525,7 +1649,7 @@ int launch_prefill_tc_local_state(int b, int T, int H, int G, const void* x, con
     prm.seg_logdecay = reinterpret_cast<float*>(static_cast<char*>(ws) + kSegOffset +
                                                 align256(units * kP * kN * sizeof(float)));
     prm.wait_ns = kWaitLimitNs;
-    SSD_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), s));
+    if ((st = reset_status(prm.status, s)) != SSD_OK) return st;
     if ((st = launch_state_pass(prm, b * H, 0, s)) != SSD_OK) return st;
     // piece q of unit u: state at (u * pieces + q) * P * N, log decay at u * pieces + q
     {

@@ -92,19 +92,19 @@ def test_long_context_sampled(L):
 
 
 def test_fused_kernel_is_the_bf16_path():
-    """bf16 with P=64, N=128 runs the fused tensor-core kernel, preceded by the segment state
-    pass and scan when the sequences are split (few sequence-heads for the SMs); other
-    shapes and fp32 run the four-kernel path."""
+    """bf16 with P=64, N=128 runs the fused tensor-core kernel after the status reset, with
+    the segment state pass between them when the sequences are split (few sequence-heads for
+    the SMs); other shapes and fp32 run the SIMT path."""
     case = make_prefill(8, 512, 80, 64, 128, 1, 256, "bf16", seed=15)
     ssd.profile_begin()
     run_prefill(ssd, case)
     kt = ssd.profile_end()
-    assert list(kt) == ["ssd_prefill_fused"] and kt["ssd_prefill_fused"][0] == 1
+    assert {k: v[0] for k, v in kt.items()} == {"ssd_status_reset": 1, "ssd_prefill_fused": 1}
     case = make_prefill(1, 4096, 24, 64, 128, 1, 256, "bf16", seed=15)  # the 130M-layer shape splits
     ssd.profile_begin()
     run_prefill(ssd, case)
     kt = ssd.profile_end()
-    assert {k: v[0] for k, v in kt.items()} == {"ssd_segment_state": 1, "ssd_segment_scan": 1,
+    assert {k: v[0] for k, v in kt.items()} == {"ssd_status_reset": 1, "ssd_segment_state": 1,
                                                  "ssd_prefill_fused": 1}
     case = make_prefill(1, 512, 4, 64, 64, 1, 256, "bf16", seed=15)
     ssd.profile_begin()
@@ -291,13 +291,19 @@ def test_bounded_wait_timeout_reports_status_and_context_survives():
     check(_np(hf), hf_ref, "bf16", "h_final after timeout")
 
 
-def test_in_place_state_resume():
-    """h_final may alias h0 exactly (in-place cache update)."""
+@pytest.mark.parametrize("nseg", [1, 4])
+def test_in_place_state_resume(nseg):
+    """h_final may alias h0 exactly (in-place cache update), also when a sequence is split
+    into segments whose CTAs run in no fixed order."""
     case = make_prefill(1, 512, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=14)
-    y, hf, t = run_prefill(ssd, case)
-    h = t["h0"].clone()
-    y2, h2 = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=256, h0=h, h_final=h)
-    torch.cuda.synchronize()
+    ssd.debug_force_prefill_segments(nseg)
+    try:
+        y, hf, t = run_prefill(ssd, case)
+        h = t["h0"].clone()
+        y2, h2 = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=256, h0=h, h_final=h)
+        torch.cuda.synchronize()
+    finally:
+        ssd.debug_force_prefill_segments(0)
     assert h2.data_ptr() == h.data_ptr()
     assert torch.equal(y2, y) and torch.equal(h, hf)
 
