@@ -24,6 +24,7 @@
 // is handled as if padded with dt = 0 tokens, which leave the state unchanged.
 #include <algorithm>
 #include <cmath>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -51,6 +52,34 @@ __device__ __forceinline__ void copy_grouped(Load load, Store store) {
         for (int k = 0; k < kGrp; ++k) r[k] = load(threadIdx.x + (k0 + k) * kThreads);
 #pragma unroll
         for (int k = 0; k < kGrp; ++k) store(threadIdx.x + (k0 + k) * kThreads, r[k]);
+    }
+}
+
+// Asynchronous 4-byte global -> shared copy (zero fill when !valid; src is then not read).
+__device__ __forceinline__ void cp_async4(float* dst, const float* src, bool valid) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
+
+// Copies a rows x W tile (row r at src_row(r), W contiguous elements; rows with !ok(r) are
+// zeros) into float shared memory with row stride `ld`: asynchronously for fp32 inputs,
+// through registers (converting) for bf16.
+template <int W, int kRows, typename RowPtr, typename RowOk>
+__device__ __forceinline__ void tile_load(float* dst, int ld, RowPtr src_row, RowOk ok) {
+    using IoT = typename std::remove_cv<typename std::remove_pointer<decltype(src_row(0))>::type>::type;
+    static_assert(kRows * W % kThreads == 0, "tile size");
+#pragma unroll
+    for (int k = 0; k < kRows * W / kThreads; ++k) {
+        const int e = threadIdx.x + k * kThreads, r = e / W, c = e % W;
+        const bool v = ok(r);
+        if constexpr (std::is_same<IoT, float>::value) {
+            cp_async4(dst + r * ld + c, v ? src_row(r) + c : src_row(0), v);
+        } else {
+            dst[r * ld + c] = v ? load_io(src_row(r), c) : 0.f;
+        }
     }
 }
 
@@ -174,8 +203,8 @@ state_scan_kernel(int T, int H, int L, int nc, int ks, const CsT* __restrict__ c
 }
 
 // ---------------------------------------------------------------- K4
-// One CTA = TR output rows (TR = 16 or 64) of one chunk of one (sequence, head); 16 x 16
-// threads, each RPT = TR / 16 rows x 4 columns (of p for the output, of j for a score tile).
+// One CTA = TR output rows of one chunk of one (sequence, head); 16 x 16 threads, each
+// RPT = TR / 16 rows x 4 columns (of p for the output, of j for a score tile).
 template <typename IoT, typename CsT, int N, int TR>
 __global__ void __launch_bounds__(kThreads)
 chunk_output_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __restrict__ x,
@@ -314,6 +343,133 @@ chunk_output_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __res
     }
 }
 
+// K4 for grids too small to fill the GPU: one CTA = 16 output rows of one chunk of one
+// (sequence, head), one row per 16 threads.  All copies are asynchronous and the column
+// tiles double-buffered: tile t + 1 is in flight while tile t is evaluated.  Same arithmetic, in the same order, as
+// chunk_output_kernel with TR = 16.
+template <typename IoT, typename CsT, int N>
+__global__ void __launch_bounds__(kThreads)
+chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __restrict__ x,
+                          const float* __restrict__ dt, const DtMap dtm, const IoT* __restrict__ Bm,
+                          const IoT* __restrict__ Cm, const float* __restrict__ D,
+                          const CsT* __restrict__ cs, const float* __restrict__ Hin,
+                          IoT* __restrict__ y) {
+    constexpr int TR = 16, TJ = 64, LD = N + 1;
+    extern __shared__ float smem[];
+    float* sC = smem;                  // [TR][LD]      C rows i
+    float* sH = sC + TR * LD;          // [kP][LD]      H_in rows p
+    float* sB = sH + kP * LD;          // [2][TJ][LD]   B rows j
+    float* sX = sB + 2 * TJ * LD;      // [2][TJ][kP]   x rows j
+    float* sG = sX + 2 * TJ * kP;      // [TR][TJ + 1]  masked decayed C.B^T
+    __shared__ CsT s_csi[TR];
+    __shared__ CsT s_csj[2][TJ];
+    __shared__ float s_dtj[2][TJ];
+
+    const int tiles_per_chunk = (L + TR - 1) / TR;
+    const int c = blockIdx.x / tiles_per_chunk, it = blockIdx.x % tiles_per_chunk;
+    const int hd = blockIdx.y, bi = blockIdx.z, g = hd / (H / G);
+    const int t0 = c * L, Lc = min(L, T - t0), i0 = it * TR;
+    if (i0 >= Lc) return;
+    const int ntile = (min(i0 + TR, Lc) + TJ - 1) / TJ;  // column tiles at and below the diagonal
+    const CsT* csc = cs + (((size_t)bi * H + hd) * nc + c) * L;
+    const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+
+    auto issue_tile = [&](int t) {  // B, x and dt of column tile t
+        const int j0 = t * TJ, buf = t & 1;
+        auto ok = [&](int j) { return j0 + j < Lc; };
+        tile_load<N, TJ>(sB + buf * TJ * LD, LD,
+                         [&](int j) { return Bm + (((size_t)bi * T + t0 + j0 + j) * G + g) * N; }, ok);
+        tile_load<kP, TJ>(sX + buf * TJ * kP, kP,
+                          [&](int j) { return x + (((size_t)bi * T + t0 + j0 + j) * H + hd) * kP; }, ok);
+        if (threadIdx.x < TJ) {
+            const int j = j0 + threadIdx.x;
+            s_dtj[buf][threadIdx.x] = j < Lc ? dt_value(dt[((size_t)bi * T + t0 + j) * H + hd], dtm, hd) : 0.f;
+        }
+    };
+    auto issue_cs = [&](int t) {  // K2's prefix sums of column tile t
+        if (threadIdx.x < TJ) {
+            const int j = t * TJ + threadIdx.x;
+            s_csj[t & 1][threadIdx.x] = j < Lc ? csc[j] : CsT(0);
+        }
+    };
+
+    // copy groups, oldest first: {C, tile 0}, {H_in}, {tile 1}, then one per loop iteration
+    tile_load<N, TR>(sC, LD, [&](int i) { return Cm + (((size_t)bi * T + t0 + i0 + i) * G + g) * N; },
+                     [&](int i) { return i0 + i < Lc; });
+    issue_tile(0);
+    cp_async_commit();
+    const float* Hc = Hin + (((size_t)bi * nc + c) * H + hd) * ks * kP * N;
+    tile_load<N, kP>(sH, LD, [&](int p) { return Hc + (size_t)p * N; }, [](int) { return true; });
+    cp_async_commit();
+    if (ntile > 1) issue_tile(1);
+    cp_async_commit();
+    if (threadIdx.x < TR) s_csi[threadIdx.x] = i0 + threadIdx.x < Lc ? csc[i0 + threadIdx.x] : CsT(0);
+    issue_cs(0);
+    if (ntile > 1) issue_cs(1);
+    cp_async_wait<1>();  // C, tile 0 and H_in landed (tile 1 may still be in flight)
+    __syncthreads();
+
+    // state-to-output term: Y[i][p] = exp(cs_i) * sum_n C[i][n] H[p][n]
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int n = 0; n < N; ++n) {
+        const float cv = sC[tr * LD + n];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] = fmaf(cv, sH[(tc * 4 + q) * LD + n], acc[q]);
+    }
+    {
+        const float e = exp_cs(s_csi[tr]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] *= e;
+    }
+
+    // intra-chunk dual form over the column tiles
+#pragma unroll 1
+    for (int t = 0; t < ntile; ++t) {
+        const int j0 = t * TJ, buf = t & 1;
+        if (t > 0) {
+            cp_async_wait<1>();  // tile t landed (tile t + 1 may be in flight)
+            __syncthreads();
+        }
+        const float* sBt = sB + buf * TJ * LD;
+        const float* sXt = sX + buf * TJ * kP;
+        float gacc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int n = 0; n < N; ++n) {
+            const float cv = sC[tr * LD + n];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) gacc[q] = fmaf(cv, sBt[(tc * 4 + q) * LD + n], gacc[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int jl = tc * 4 + q;
+            float v = 0.f;
+            if (j0 + jl <= i0 + tr) v = gacc[q] * exp_cs(s_csi[tr] - s_csj[buf][jl]) * s_dtj[buf][jl];
+            sG[tr * (TJ + 1) + jl] = v;
+        }
+        __syncthreads();
+        for (int j = 0; j < TJ; ++j) {
+            const float gv = sG[tr * (TJ + 1) + j];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] = fmaf(gv, sXt[j * kP + tc * 4 + q], acc[q]);
+        }
+        __syncthreads();  // buffers of tile t and the score tile are free
+        if (t + 2 < ntile) {
+            issue_tile(t + 2);
+            issue_cs(t + 2);
+        }
+        cp_async_commit();
+    }
+    const int i = i0 + tr;
+    if (i < Lc) {
+        const float Dv = D[hd];
+        const size_t off = (((size_t)bi * T + t0 + i) * H + hd) * kP;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int p = tc * 4 + q;
+            store_io(y, off + p, acc[q] + Dv * load_io(x, off + p));
+        }
+    }
+}
+
 int sm_count_simt() {
     static int n = 0;
     if (n <= 0) {
@@ -337,11 +493,16 @@ int state_slices(int b, int T, int H, int N, int L) {
     return ks;
 }
 
-template <typename IoT, typename CsT, int N, int TR>
+// K4: 64-row tiles, or the pipelined 16-row kernel when 64-row tiles would not give every
+// SM two CTAs
+template <typename IoT, typename CsT, int N>
 int launch_output(int b, int T, int H, int G, int L, int nc, int ks, const IoT* x, const float* dt, const DtMap& dtm,
                   const IoT* Bm, const IoT* Cm, const float* D, const CsT* cs, const float* S, void* y, cudaStream_t s) {
-    const size_t smem = sizeof(float) * (TR * (N + 1) + 64 * (N + 1) + TR * 65 + 64 * kP);
-    auto k4 = chunk_output_kernel<IoT, CsT, N, TR>;
+    const bool small = (double)nc * ((L + 63) / 64) * H * b < 2.0 * sm_count_simt();
+    const int TR = small ? 16 : 64;
+    const size_t smem = small ? sizeof(float) * (16 * (N + 1) + kP * (N + 1) + 2 * 64 * (N + 1) + 2 * 64 * kP + 16 * 65)
+                              : sizeof(float) * (64 * (N + 1) + 64 * (N + 1) + 64 * 65 + 64 * kP);
+    auto k4 = small ? chunk_output_small_kernel<IoT, CsT, N> : chunk_output_kernel<IoT, CsT, N, 64>;
     if (const int st = smem_limit_once((const void*)k4, (int)smem)) return st;
     LaunchScope ls("simt_chunk_output", s);
     k4<<<dim3(nc * ((L + TR - 1) / TR), H, b), kThreads, smem, s>>>(T, H, G, L, nc, ks, x, dt, dtm, Bm, Cm, D, cs, S,
@@ -369,10 +530,7 @@ int run(int b, int T, int H, int G, int L, const void* x, const float* dt, const
         LaunchScope ls("simt_state_scan", s);
         state_scan_kernel<CsT, N><<<dim3(kP * N / kThreads, H, b), kThreads, 0, s>>>(T, H, L, nc, ks, cs, h0, S, hf);
     }
-    // 16-row output tiles when 64-row tiles would not give every SM two CTAs
-    const bool small = (double)nc * ((L + 63) / 64) * H * b < 2.0 * sm_count_simt();
-    const int st = small ? launch_output<IoT, CsT, N, 16>(b, T, H, G, L, nc, ks, xi, dt, dtm, Bi, Ci, D, cs, S, y, s)
-                         : launch_output<IoT, CsT, N, 64>(b, T, H, G, L, nc, ks, xi, dt, dtm, Bi, Ci, D, cs, S, y, s);
+    const int st = launch_output<IoT, CsT, N>(b, T, H, G, L, nc, ks, xi, dt, dtm, Bi, Ci, D, cs, S, y, s);
     if (st != SSD_OK) return st;
     SSD_CUDA_TRY(cudaGetLastError());
     return SSD_OK;
