@@ -65,9 +65,9 @@ template <int kPending>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
 
 // Copies a rows x W tile (row r at src_row(r), W contiguous elements; rows with !ok(r) are
-// zeros) into float shared memory with row stride `ld`: asynchronously for fp32 inputs,
-// through registers (converting) for bf16.
-template <int W, int kRows, typename RowPtr, typename RowOk>
+// zeros) into float shared memory, element (r, c) at dst[r * ld + c] or, transposed, at
+// dst[c * ld + r]: asynchronously for fp32 inputs, through registers (converting) for bf16.
+template <int W, int kRows, bool kTransposed, typename RowPtr, typename RowOk>
 __device__ __forceinline__ void tile_load(float* dst, int ld, RowPtr src_row, RowOk ok) {
     using IoT = typename std::remove_cv<typename std::remove_pointer<decltype(src_row(0))>::type>::type;
     static_assert(kRows * W % kThreads == 0, "tile size");
@@ -75,10 +75,11 @@ __device__ __forceinline__ void tile_load(float* dst, int ld, RowPtr src_row, Ro
     for (int k = 0; k < kRows * W / kThreads; ++k) {
         const int e = threadIdx.x + k * kThreads, r = e / W, c = e % W;
         const bool v = ok(r);
+        float* d = kTransposed ? dst + c * ld + r : dst + r * ld + c;
         if constexpr (std::is_same<IoT, float>::value) {
-            cp_async4(dst + r * ld + c, v ? src_row(r) + c : src_row(0), v);
+            cp_async4(d, v ? src_row(r) + c : src_row(0), v);
         } else {
-            dst[r * ld + c] = v ? load_io(src_row(r), c) : 0.f;
+            *d = v ? load_io(src_row(r), c) : 0.f;
         }
     }
 }
@@ -107,6 +108,23 @@ chunk_state_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __rest
     __shared__ float sX[KT][kP];
     __shared__ float sB[KT][N];
     __shared__ float sW[KT];
+    // x and B of a stage are loaded into registers one stage ahead (the first before the
+    // prefix sums), so their latency overlaps the scan and the previous stage's products
+    constexpr int XR = KT * kP / kThreads, BR = KT * N / kThreads;
+    float xr[XR], br[BR];
+    auto load_stage = [&](int k0) {
+#pragma unroll
+        for (int k = 0; k < XR; ++k) {
+            const int e = threadIdx.x + k * kThreads, t = k0 + e / kP;
+            xr[k] = t < Lc ? load_io(x, (((size_t)bi * T + t0 + t) * H + hd) * kP + e % kP) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < BR; ++k) {
+            const int e = threadIdx.x + k * kThreads, t = k0 + e / N;
+            br[k] = t < Lc ? load_io(Bm, (((size_t)bi * T + t0 + t) * G + g) * N + e % N) : 0.f;
+        }
+    };
+    load_stage(sl * KT);
     {
         // inclusive prefix sum of a = dt*A over the chunk (tokens past its end add 0)
         const int j = threadIdx.x, lane = j & 31, w = j >> 5;
@@ -138,19 +156,18 @@ chunk_state_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __rest
             sW[threadIdx.x] = t < Lc ? exp_cs(cs_last - s_cs[t]) * dt_value(dt[((size_t)bi * T + t0 + t) * H + hd], dtm, hd) : 0.f;
         }
         __syncthreads();
-        copy_grouped<KT * kP>(
-            [&](int e) {
-                const int t = k0 + e / kP;
-                return t < Lc ? load_io(x, (((size_t)bi * T + t0 + t) * H + hd) * kP + e % kP) : 0.f;
-            },
-            [&](int e, float v) { sX[e / kP][e % kP] = sW[e / kP] * v; });
-        copy_grouped<KT * N>(
-            [&](int e) {
-                const int t = k0 + e / N;
-                return t < Lc ? load_io(Bm, (((size_t)bi * T + t0 + t) * G + g) * N + e % N) : 0.f;
-            },
-            [&](int e, float v) { sB[e / N][e % N] = v; });
+#pragma unroll
+        for (int k = 0; k < XR; ++k) {
+            const int e = threadIdx.x + k * kThreads;
+            sX[e / kP][e % kP] = sW[e / kP] * xr[k];
+        }
+#pragma unroll
+        for (int k = 0; k < BR; ++k) {
+            const int e = threadIdx.x + k * kThreads;
+            sB[e / N][e % N] = br[k];
+        }
         __syncthreads();
+        if (k0 + ks * KT < Lc) load_stage(k0 + ks * KT);
 #pragma unroll 4
         for (int j = 0; j < KT; ++j) {
             float xv[PR], bv[8];
@@ -344,9 +361,21 @@ chunk_output_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __res
 }
 
 // K4 for grids too small to fill the GPU: one CTA = 16 output rows of one chunk of one
-// (sequence, head), one row per 16 threads.  All copies are asynchronous and the column
-// tiles double-buffered: tile t + 1 is in flight while tile t is evaluated.  Same arithmetic, in the same order, as
-// chunk_output_kernel with TR = 16.
+// (sequence, head); thread (row, group of four columns).  B and H_in are kept transposed
+// ([n][j], [n][p]) and x row-major, so that every step of the three products reads the
+// thread's four columns with one 16-byte shared load beside one broadcast value (these
+// small grids are bound by shared-memory issue, not by arithmetic).  All copies are
+// asynchronous into a ring of kDepth column tiles (the whole 256-token chunk at N = 64), so
+// up to kDepth - 1 tiles are in flight while one is evaluated.  Same arithmetic, in the same
+// order, as chunk_output_kernel.
+constexpr int kSmallRows = 16, kSmallCols = 64, kLdT = 68;  // transposed rows: 64 + 4 (16-byte aligned)
+template <int N>
+constexpr int small_depth() { return N == 64 ? 4 : 2; }
+template <int N>
+constexpr size_t small_smem_bytes() {
+    return sizeof(float) * (kSmallRows * (N + 1) + N * kLdT + small_depth<N>() * (N * kLdT + kSmallCols * kP) +
+                            kSmallRows * (kSmallCols + 1));
+}
 template <typename IoT, typename CsT, int N>
 __global__ void __launch_bounds__(kThreads)
 chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __restrict__ x,
@@ -354,16 +383,17 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
                           const IoT* __restrict__ Cm, const float* __restrict__ D,
                           const CsT* __restrict__ cs, const float* __restrict__ Hin,
                           IoT* __restrict__ y) {
-    constexpr int TR = 16, TJ = 64, LD = N + 1;
-    extern __shared__ float smem[];
-    float* sC = smem;                  // [TR][LD]      C rows i
-    float* sH = sC + TR * LD;          // [kP][LD]      H_in rows p
-    float* sB = sH + kP * LD;          // [2][TJ][LD]   B rows j
-    float* sX = sB + 2 * TJ * LD;      // [2][TJ][kP]   x rows j
-    float* sG = sX + 2 * TJ * kP;      // [TR][TJ + 1]  masked decayed C.B^T
+    constexpr int TR = kSmallRows, TJ = kSmallCols, LD = N + 1, kDepth = small_depth<N>();
+    static_assert(TJ == kP && TR * 16 == kThreads, "thread (row, four columns of j and of p)");
+    extern __shared__ __align__(16) float smem[];
+    float* sC = smem;                     // [TR][LD]            C rows i
+    float* sHT = sC + TR * LD;            // [N][kLdT]           H_in, transposed: [n][p]
+    float* sBT = sHT + N * kLdT;          // [kDepth][N][kLdT]   B, transposed: [n][j]
+    float* sX = sBT + kDepth * N * kLdT;  // [kDepth][TJ][kP]    x rows j
+    float* sG = sX + kDepth * TJ * kP;    // [TR][TJ + 1]        masked decayed C.B^T
     __shared__ CsT s_csi[TR];
-    __shared__ CsT s_csj[2][TJ];
-    __shared__ float s_dtj[2][TJ];
+    __shared__ CsT s_csj[kDepth][TJ];
+    __shared__ float s_dtj[kDepth][TJ];
 
     const int tiles_per_chunk = (L + TR - 1) / TR;
     const int c = blockIdx.x / tiles_per_chunk, it = blockIdx.x % tiles_per_chunk;
@@ -372,49 +402,52 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
     if (i0 >= Lc) return;
     const int ntile = (min(i0 + TR, Lc) + TJ - 1) / TJ;  // column tiles at and below the diagonal
     const CsT* csc = cs + (((size_t)bi * H + hd) * nc + c) * L;
-    const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+    const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;  // row i0 + tr, columns 4 tc .. 4 tc + 3
 
-    auto issue_tile = [&](int t) {  // B, x and dt of column tile t
-        const int j0 = t * TJ, buf = t & 1;
+    auto issue_tile = [&](int t) {  // B, x, dt and the prefix sums of column tile t into slot t % kDepth
+        if (t >= ntile) return;
+        const int j0 = t * TJ, buf = t % kDepth;
         auto ok = [&](int j) { return j0 + j < Lc; };
-        tile_load<N, TJ>(sB + buf * TJ * LD, LD,
-                         [&](int j) { return Bm + (((size_t)bi * T + t0 + j0 + j) * G + g) * N; }, ok);
-        tile_load<kP, TJ>(sX + buf * TJ * kP, kP,
-                          [&](int j) { return x + (((size_t)bi * T + t0 + j0 + j) * H + hd) * kP; }, ok);
+        tile_load<N, TJ, true>(sBT + buf * N * kLdT, kLdT,
+                               [&](int j) { return Bm + (((size_t)bi * T + t0 + j0 + j) * G + g) * N; }, ok);
+        tile_load<kP, TJ, false>(sX + buf * TJ * kP, kP,
+                                 [&](int j) { return x + (((size_t)bi * T + t0 + j0 + j) * H + hd) * kP; }, ok);
         if (threadIdx.x < TJ) {
             const int j = j0 + threadIdx.x;
             s_dtj[buf][threadIdx.x] = j < Lc ? dt_value(dt[((size_t)bi * T + t0 + j) * H + hd], dtm, hd) : 0.f;
-        }
-    };
-    auto issue_cs = [&](int t) {  // K2's prefix sums of column tile t
-        if (threadIdx.x < TJ) {
-            const int j = t * TJ + threadIdx.x;
-            s_csj[t & 1][threadIdx.x] = j < Lc ? csc[j] : CsT(0);
+            s_csj[buf][threadIdx.x] = j < Lc ? csc[j] : CsT(0);
         }
     };
 
-    // copy groups, oldest first: {C, tile 0}, {H_in}, {tile 1}, then one per loop iteration
-    tile_load<N, TR>(sC, LD, [&](int i) { return Cm + (((size_t)bi * T + t0 + i0 + i) * G + g) * N; },
-                     [&](int i) { return i0 + i < Lc; });
+    // copy groups, oldest first: {C, tile 0}, {H_in}, {tile 1} .. {tile kDepth - 1}, then one
+    // per loop iteration (empty where there is no tile), so that tile t is complete once at
+    // most kDepth - 1 groups are pending
+    tile_load<N, TR, false>(sC, LD, [&](int i) { return Cm + (((size_t)bi * T + t0 + i0 + i) * G + g) * N; },
+                            [&](int i) { return i0 + i < Lc; });
     issue_tile(0);
     cp_async_commit();
     const float* Hc = Hin + (((size_t)bi * nc + c) * H + hd) * ks * kP * N;
-    tile_load<N, kP>(sH, LD, [&](int p) { return Hc + (size_t)p * N; }, [](int) { return true; });
+    tile_load<N, kP, true>(sHT, kLdT, [&](int p) { return Hc + (size_t)p * N; }, [](int) { return true; });
     cp_async_commit();
-    if (ntile > 1) issue_tile(1);
-    cp_async_commit();
+#pragma unroll
+    for (int t = 1; t < kDepth; ++t) {
+        issue_tile(t);
+        cp_async_commit();
+    }
     if (threadIdx.x < TR) s_csi[threadIdx.x] = i0 + threadIdx.x < Lc ? csc[i0 + threadIdx.x] : CsT(0);
-    issue_cs(0);
-    if (ntile > 1) issue_cs(1);
-    cp_async_wait<1>();  // C, tile 0 and H_in landed (tile 1 may still be in flight)
+    cp_async_wait<kDepth - 1>();  // C, tile 0 and H_in landed
     __syncthreads();
 
     // state-to-output term: Y[i][p] = exp(cs_i) * sum_n C[i][n] H[p][n]
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
     for (int n = 0; n < N; ++n) {
         const float cv = sC[tr * LD + n];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[q] = fmaf(cv, sH[(tc * 4 + q) * LD + n], acc[q]);
+        const float4 h4 = *reinterpret_cast<const float4*>(sHT + n * kLdT + 4 * tc);
+        acc[0] = fmaf(cv, h4.x, acc[0]);
+        acc[1] = fmaf(cv, h4.y, acc[1]);
+        acc[2] = fmaf(cv, h4.z, acc[2]);
+        acc[3] = fmaf(cv, h4.w, acc[3]);
     }
     {
         const float e = exp_cs(s_csi[tr]);
@@ -425,37 +458,42 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
     // intra-chunk dual form over the column tiles
 #pragma unroll 1
     for (int t = 0; t < ntile; ++t) {
-        const int j0 = t * TJ, buf = t & 1;
+        const int j0 = t * TJ, buf = t % kDepth;
         if (t > 0) {
-            cp_async_wait<1>();  // tile t landed (tile t + 1 may be in flight)
+            cp_async_wait<kDepth - 1>();  // tile t landed
             __syncthreads();
         }
-        const float* sBt = sB + buf * TJ * LD;
+        const float* sBt = sBT + buf * N * kLdT;
         const float* sXt = sX + buf * TJ * kP;
         float gacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
         for (int n = 0; n < N; ++n) {
             const float cv = sC[tr * LD + n];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) gacc[q] = fmaf(cv, sBt[(tc * 4 + q) * LD + n], gacc[q]);
+            const float4 b4 = *reinterpret_cast<const float4*>(sBt + n * kLdT + 4 * tc);
+            gacc[0] = fmaf(cv, b4.x, gacc[0]);
+            gacc[1] = fmaf(cv, b4.y, gacc[1]);
+            gacc[2] = fmaf(cv, b4.z, gacc[2]);
+            gacc[3] = fmaf(cv, b4.w, gacc[3]);
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int jl = tc * 4 + q;
+            const int jl = 4 * tc + q;
             float v = 0.f;
             if (j0 + jl <= i0 + tr) v = gacc[q] * exp_cs(s_csi[tr] - s_csj[buf][jl]) * s_dtj[buf][jl];
             sG[tr * (TJ + 1) + jl] = v;
         }
         __syncthreads();
+#pragma unroll 4
         for (int j = 0; j < TJ; ++j) {
             const float gv = sG[tr * (TJ + 1) + j];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc[q] = fmaf(gv, sXt[j * kP + tc * 4 + q], acc[q]);
+            const float4 x4 = *reinterpret_cast<const float4*>(sXt + j * kP + 4 * tc);
+            acc[0] = fmaf(gv, x4.x, acc[0]);
+            acc[1] = fmaf(gv, x4.y, acc[1]);
+            acc[2] = fmaf(gv, x4.z, acc[2]);
+            acc[3] = fmaf(gv, x4.w, acc[3]);
         }
-        __syncthreads();  // buffers of tile t and the score tile are free
-        if (t + 2 < ntile) {
-            issue_tile(t + 2);
-            issue_cs(t + 2);
-        }
+        __syncthreads();  // slot t % kDepth and the score tile are free
+        issue_tile(t + kDepth);
         cp_async_commit();
     }
     const int i = i0 + tr;
@@ -464,7 +502,7 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
         const size_t off = (((size_t)bi * T + t0 + i) * H + hd) * kP;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int p = tc * 4 + q;
+            const int p = 4 * tc + q;
             store_io(y, off + p, acc[q] + Dv * load_io(x, off + p));
         }
     }
@@ -499,9 +537,8 @@ template <typename IoT, typename CsT, int N>
 int launch_output(int b, int T, int H, int G, int L, int nc, int ks, const IoT* x, const float* dt, const DtMap& dtm,
                   const IoT* Bm, const IoT* Cm, const float* D, const CsT* cs, const float* S, void* y, cudaStream_t s) {
     const bool small = (double)nc * ((L + 63) / 64) * H * b < 2.0 * sm_count_simt();
-    const int TR = small ? 16 : 64;
-    const size_t smem = small ? sizeof(float) * (16 * (N + 1) + kP * (N + 1) + 2 * 64 * (N + 1) + 2 * 64 * kP + 16 * 65)
-                              : sizeof(float) * (64 * (N + 1) + 64 * (N + 1) + 64 * 65 + 64 * kP);
+    const int TR = small ? kSmallRows : 64;
+    const size_t smem = small ? small_smem_bytes<N>() : sizeof(float) * (64 * (N + 1) + 64 * (N + 1) + 64 * 65 + 64 * kP);
     auto k4 = small ? chunk_output_small_kernel<IoT, CsT, N> : chunk_output_kernel<IoT, CsT, N, 64>;
     if (const int st = smem_limit_once((const void*)k4, (int)smem)) return st;
     LaunchScope ls("simt_chunk_output", s);
