@@ -567,6 +567,8 @@ def main():
                 "hbm_gbs_alg": pbytes * world / (ms * 1e-3) / 1e9,
                 "tensor_frac": tflops / world / pk["bf16_tflops"],
                 "gpu_launches_all_timed_regions": int(launches),
+                "prefill_split": {"whole_units": ssd.prefill_whole_units(PB, PT, PH, PP, PN, PG, PL, ssd.SSD_BF16),
+                                  "segments": ssd.prefill_segments(PB, PT, PH, PP, PN, PG, PL, ssd.SSD_BF16)},
                 "clocks": clk, "decode": decode, "prefill_configs": other, "prefill_dt_raw": dt_raw_entry,
                 "decay_precision_ablation": ablation}
         print(json.dumps(line), flush=True)

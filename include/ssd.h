@@ -216,10 +216,18 @@ SSD_API int ssd_debug_decay_precision(int mode);
 
 /* Segments per sequence that ssd_prefill would use for this shape: 1 when the whole
  * sequence runs in one pass (every shape outside the tensor-core path, and tensor-core
- * shapes with enough sequence-heads for the SMs of the current device), else the count of
- * 128-token-aligned segments (see ssd_prefill: local end states, a scan, then the fused
- * pass per segment).  Returns 0 for an invalid shape.  Host-only; nothing is enqueued. */
+ * shapes whose sequence-heads fill the SMs of the current device in whole waves), else the
+ * count of 128-token-aligned segments of each split sequence-head (see ssd_prefill: local
+ * end states, then the fused pass per segment, which folds the earlier segments' states).
+ * Returns 0 for an invalid shape.  Host-only; nothing is enqueued. */
 SSD_API int ssd_prefill_segments(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype);
+
+/* How many (sequence, head) pairs ssd_prefill runs whole, in one pass each, for this
+ * shape: b*H when nothing is split, 0 when every pair is split into
+ * ssd_prefill_segments(...) segments, or the pairs of the whole waves of CTAs when only the
+ * pairs of a ragged last wave are split (pairs are ordered bi * H + head).  Returns -1 for
+ * an invalid shape.  Host-only; nothing is enqueued. */
+SSD_API int ssd_prefill_whole_units(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype);
 
 /* ------------------------------------------------------------------------------------
  * Cached decode step  ([CF-SSD] O(1) caching section)

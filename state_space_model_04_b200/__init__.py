@@ -29,6 +29,7 @@ from .ssd import (  # noqa: F401
     prefill_context_scan,
     prefill_local_state,
     prefill_segments,
+    prefill_whole_units,
     prefill_workspace_size,
     status_string,
 )

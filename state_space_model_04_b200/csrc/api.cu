@@ -34,6 +34,7 @@ void prefill_tc_force_segments(int nseg);
 void prefill_tc_force_split(int n_full, int nseg);
 void prefill_tc_decay_mode(int mode);
 int prefill_tc_segments(int b, int T, int H);
+int prefill_tc_whole_units(int b, int T, int H);
 size_t prefill_tc_local_state_workspace_bytes(int b, int T, int H);
 int launch_prefill_tc_local_state(int b, int T, int H, int G, const void* x, const float* dt, const float* A,
                                   const void* Bm, float* h_local, float* log_decay, void* ws, cudaStream_t s);
@@ -246,6 +247,12 @@ int ssd_prefill_segments(int b, int T, int H, int P, int N, int G, int chunk, in
     if (check_prefill_shape(b, T, H, P, N, G, chunk, io_dtype) != SSD_OK) return 0;
     if (b == 0 || T == 0 || !prefill_tc_supported(P, N, io_dtype)) return 1;
     return prefill_tc_segments(b, T, H);
+}
+
+int ssd_prefill_whole_units(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype) {
+    if (check_prefill_shape(b, T, H, P, N, G, chunk, io_dtype) != SSD_OK) return -1;
+    if (b == 0 || T == 0 || !prefill_tc_supported(P, N, io_dtype)) return b * H;
+    return prefill_tc_whole_units(b, T, H);
 }
 
 size_t ssd_prefill_local_state_workspace_size(int b, int T, int H, int P, int N, int G, int io_dtype) {

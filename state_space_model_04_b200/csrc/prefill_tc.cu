@@ -1427,9 +1427,13 @@ int sm_count() {
 // allocation, first loads) costs about two more block-times.  Splitting units into
 // segments adds CTAs where b * H alone leaves SMs idle -- all units when b * H is below
 // the SM count, or only the units of a ragged last wave -- at the price of the state pass
-// (two CTAs per SM, measured at about 0.7 of a fused block-time per block), the scan
-// (about 0.4 block-times per segment) and a fixed cost for the two extra launches.  No
-// split wherever the split does not pay by 5 %.
+// (two CTAs per SM, measured at about 0.7 of a fused block-time per block), the fold of the
+// segment states (about 0.4 block-times per segment) and a fixed cost for the extra launch.
+// The cheapest candidate wins, but only where it beats the unsplit pass by 5 %.  Splitting only the units of a ragged
+// last wave is priced from its own measurements instead: the state pass then runs beside
+// the first wave of whole units (the fused grid may start as soon as the state pass runs),
+// and costs about 1.5 block-times per extra segment plus one; that split is taken when it
+// pays by 3 %.
 struct SplitPlan {
     int n_full, nseg, tseg;  // see TcParams
 };
@@ -1437,6 +1441,7 @@ constexpr double kStatePassPerBlock = 0.7;  // single-head state pass; the paire
 constexpr double kCtaStartBlocks = 2.0;
 constexpr double kScanPerSegment = 0.4;
 constexpr double kSplitFixedBlocks = 5.0;
+constexpr double kTailSplitPerSegment = 1.5, kTailSplitFixed = 1.0;
 constexpr int kFoldMax = 5;  // the fused kernel folds up to this many segment states itself
 std::atomic<int> g_force_nseg{0};     // 0: cost model
 std::atomic<int> g_force_nfull{-1};   // -1: every unit split when nseg > 1
@@ -1473,12 +1478,16 @@ SplitPlan plan_split(int b, int T, int H) {
         const double r = units - n_full;
         for (int bps = nb - 1; bps >= 1; --bps) {
             const int n = (nb + bps - 1) / bps;
-            if ((nb + bps) / (bps + 1) == n) continue;  // same segment count as a longer bps
+            // of the lengths that give n segments only the shortest (the most even split) counts
+            if (bps > 1 && (nb + bps - 2) / (bps - 1) == n) continue;
             const double len = bps + kCtaStartBlocks;
             double cost = (n_full ? std::ceil(n_full / sms) * (nb + kCtaStartBlocks) : 0.0) + pass_cost(r * n, len, sms);
-            cost += kStatePassPerBlock * std::ceil(r * (n - 1) / (2.0 * sms)) * len + kScanPerSegment * n +
-                    kSplitFixedBlocks;
-            if (cost < 0.95 * best_cost) {
+            if (n_full)
+                cost += kTailSplitPerSegment * (n - 1) + kTailSplitFixed;
+            else
+                cost += kStatePassPerBlock * std::ceil(r * (n - 1) / (2.0 * sms)) * len + kScanPerSegment * n +
+                        kSplitFixedBlocks;
+            if (cost < (n_full ? 0.97 : 0.95) * whole && cost < best_cost) {
                 best_cost = cost;
                 best = SplitPlan{n_full, n, bps * kBlk};
             }
@@ -1489,6 +1498,10 @@ SplitPlan plan_split(int b, int T, int H) {
 }  // namespace
 
 int prefill_tc_segments(int b, int T, int H) { return plan_split(b, T, H).nseg; }
+int prefill_tc_whole_units(int b, int T, int H) {
+    const SplitPlan sp = plan_split(b, T, H);
+    return sp.nseg == 1 ? b * H : sp.n_full;
+}
 
 // Workspace: the status word, then (split sequences only) the segments' end states, their
 // log decays, and room for a copy of the split units' h0.

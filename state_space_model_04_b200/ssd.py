@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_prefill_context_scan.restype = _i
         L.ssd_prefill_segments.argtypes = [_i] * 8
         L.ssd_prefill_segments.restype = _i
+        L.ssd_prefill_whole_units.argtypes = [_i] * 8
+        L.ssd_prefill_whole_units.restype = _i
         L.ssd_debug_decay_precision.argtypes = [_i]
         L.ssd_debug_decay_precision.restype = _i
         L.ssd_debug_force_prefill_split.argtypes = [_i, _i]
@@ -270,6 +272,12 @@ def prefill_context_scan(rank, h_local_all, log_decay_all, h0=None, h_in=None, s
 def prefill_segments(b, T, H, P, N, G, chunk, io_dtype) -> int:
     """Segments per sequence ssd_prefill uses for this shape (1 = one pass; 0 = invalid)."""
     return int(lib().ssd_prefill_segments(b, T, H, P, N, G, chunk, io_dtype))
+
+
+def prefill_whole_units(b, T, H, P, N, G, chunk, io_dtype) -> int:
+    """(Sequence, head) pairs ssd_prefill runs whole for this shape (-1 = invalid); the rest
+    are split into prefill_segments(...) segments each."""
+    return int(lib().ssd_prefill_whole_units(b, T, H, P, N, G, chunk, io_dtype))
 
 
 def debug_decay_precision(mode=0):

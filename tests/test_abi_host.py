@@ -172,9 +172,16 @@ def test_segment_hook_and_workspace():
     assert ssd.lib().ssd_debug_force_prefill_segments(-1) == 1  # SSD_ERR_INVALID_ARG
     try:
         assert ssd.prefill_segments(*args) >= 1
-        assert ssd.prefill_segments(8, 4096, 80, 64, 128, 1, 256, 1) == 1   # enough sequence-heads
+        assert ssd.prefill_whole_units(*args) == 0                            # every pair split
+        assert ssd.prefill_segments(16, 4096, 80, 64, 128, 1, 256, 1) == 1  # enough sequence-heads
+        assert ssd.prefill_whole_units(16, 4096, 80, 64, 128, 1, 256, 1) == 16 * 80
+        # 640 pairs on 148 SMs: the 48 pairs of the ragged last wave are split, the rest run whole
+        assert ssd.prefill_segments(8, 4096, 80, 64, 128, 1, 256, 1) > 1
+        assert ssd.prefill_whole_units(8, 4096, 80, 64, 128, 1, 256, 1) in (0, 592)
         assert ssd.prefill_segments(1, 4096, 24, 64, 64, 1, 256, 1) == 1    # N = 64: the SIMT path
+        assert ssd.prefill_whole_units(1, 4096, 24, 64, 64, 1, 256, 1) == 24
         assert ssd.prefill_segments(1, 512, 4, 64, 64, 1, 100, 0) == 0      # invalid chunk
+        assert ssd.prefill_whole_units(1, 512, 4, 64, 64, 1, 100, 0) == -1
         ssd.debug_force_prefill_segments(1)
         assert ssd.prefill_segments(*args) == 1
         one = ssd.prefill_workspace_size(*args)
