@@ -614,9 +614,9 @@ def bench_prefill_configs(ssd, torch, dev, stream, args, clocks, barrier, max_ov
     long-context shape (b=1, T=65536, H=80, G=8), inputs resident in HBM, each step timed
     alone with CUDA events on the launching stream after a write that evicts L2, max over
     ranks; the per-kernel times come from a second pass with events around every launch.  The fused tensor-core path
-    evaluates 128-token chunks whatever chunk length is requested, so the long-context
-    configuration's chunk-length sweep is one decomposition: it is timed once and reported
-    with chunk_executed = 128 and the operation count of that decomposition.  The bf16
+    evaluates 128-token chunks whatever chunk length is requested: the long-context entry is
+    timed once on it (chunk_executed = 128), and its chunk-length sweep L in {64, 128, 256}
+    is timed literally on the fp32-FMA path (literal_chunk_sweep).  The bf16
     shapes have few (sequence, head) pairs for 148 SMs, so their sequences are split into
     segments (state pass, a prefix pass when there are many segments, fused pass); the
     segment count is reported."""
@@ -678,9 +678,53 @@ def bench_prefill_configs(ssd, torch, dev, stream, args, clocks, barrier, max_ov
                  "kernels": {k: {"launches": v[0] // n_steps, "avg_ms": v[1] / max(v[0], 1)} for k, v in kt.items()},
                  "segments": ssd.prefill_segments(b, T, H, P, N, G, 256, io),
                  "l2": "256 MB written before every timed step"}
+        if label == "long_context":
+            entry["literal_chunk_sweep"] = literal_chunk_sweep(ssd, torch, x, dt, A, Bm, Cm, D, y, hfin, flush,
+                                                               stream, barrier, max_over_ranks, world, box,
+                                                               (b, T, H, P, N, G))
         out[label] = entry
         del x, Bm, Cm, dt, A, D, y, hfin, ws
         torch.cuda.empty_cache()
+    return out
+
+
+def literal_chunk_sweep(ssd, torch, x, dt, A, Bm, Cm, D, y, hfin, flush, stream, barrier, max_over_ranks, world,
+                        box, shape):
+    """The long-context prefill with chunks of exactly L tokens for L in {64, 128, 256}: the
+    fp32-FMA path (ssd_debug_force_fma_prefill) evaluates the chunked form with the chunk
+    length given, so this is the pages' chunk-size trade-off (arithmetic intensity of the
+    dual form against the length of the sequential recurrence) measured on kernels that
+    honour L.  The tensor-core kernel always evaluates 128-token chunks (its timing is the
+    entry's ms_per_step).  Each L: one warm-up call, then two calls timed alone after an
+    L2-evicting write; ms per call and TFLOP/s at that L's operation count."""
+    b, T, H, P, N, G = shape
+    out = {"path": "fp32 FMA (SIMT), bf16 io, literal chunk length"}
+    ssd.debug_force_fma_prefill(True)
+    try:
+        for L in (64, 128, 256):
+            ws = torch.empty(ssd.prefill_workspace_size(b, T, H, P, N, G, L, ssd.SSD_BF16), dtype=torch.uint8,
+                             device=x.device)
+            def step():
+                ssd.prefill(x, dt, A, Bm, Cm, D, chunk=L, y=y, h_final=hfin, workspace=ws)
+            step()
+            torch.cuda.synchronize()
+            barrier()
+            n0 = ssd.launch_count()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
+            for ev in evs:
+                flush.fill_(1)
+                ev[0].record(stream)
+                step()
+                ev[1].record(stream)
+            torch.cuda.synchronize()
+            box[0] += ssd.launch_count() - n0
+            ms = max_over_ranks(sum(a.elapsed_time(c) for a, c in evs) / len(evs))
+            out["L%d" % L] = {"ms_per_step": ms,
+                              "tflops": job_rate(prefill_flops(b, T, H, P, N, G, L), world, ms) / 1e12}
+            del ws
+            torch.cuda.empty_cache()
+    finally:
+        ssd.debug_force_fma_prefill(False)
     return out
 
 

@@ -193,7 +193,7 @@ SSD_API int ssd_debug_starve_next_prefill(unsigned long long wait_limit_ns);
  * splits each sequence into min(nseg, ceil(T / 128)) segments of whole 128-token blocks
  * instead of the count its cost model picks; nseg = 0 restores the cost model.  The
  * result is the same function either way (only rounding differs): segments after the
- * first start from the state a scan of the earlier segments' local end states gives.
+ * first start from the fold of the earlier segments' local end states.
  * Not thread-safe against concurrent prefill calls.
  * Errors: SSD_ERR_INVALID_ARG if nseg < 0. */
 SSD_API int ssd_debug_force_prefill_segments(int nseg);
@@ -203,6 +203,17 @@ SSD_API int ssd_debug_force_prefill_segments(int nseg);
  * cost model's "ragged last wave" split).  n_full is clamped to b * H; nseg = 0 restores
  * the cost model.  Errors: SSD_ERR_INVALID_ARG if n_full < 0 or nseg < 0. */
 SSD_API int ssd_debug_force_prefill_split(int n_full, int nseg);
+
+/* Test and measurement hook: with on = 1, every following ssd_prefill / ssd_prefill_dt_raw
+ * in this process (and ssd_prefill_workspace_size, ssd_prefill_segments,
+ * ssd_prefill_whole_units) takes the fp32-FMA path even for shapes the tensor-core kernel
+ * takes.  That path evaluates the chunked dual form with chunks of exactly `chunk` tokens,
+ * so it serves the literal chunk-length sweep ([CF-SSD] "Chunked recurrence": the chunk
+ * size trades arithmetic intensity against sequential overhead) at any shape; it is an
+ * order of magnitude slower than the tensor-core kernel.  on = 0 restores the default.
+ * Not thread-safe against concurrent prefill calls.
+ * Errors: SSD_ERR_INVALID_ARG if on is not 0 or 1. */
+SSD_API int ssd_debug_force_fma_prefill(int on);
 
 /* Decay-precision ablation for the tensor-core prefill ([CF-SSD] "Precision management":
  * decay parameters held in log space in fp32 and exponentiated at compute time; bf16 for

@@ -12,6 +12,7 @@ from .ssd import (  # noqa: F401
     DecodePlan,
     SSDError,
     debug_decay_precision,
+    debug_force_fma_prefill,
     debug_force_prefill_segments,
     debug_force_prefill_split,
     debug_starve_next_prefill,

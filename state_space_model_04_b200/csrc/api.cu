@@ -224,8 +224,12 @@ int ssd_profile_end(ssd_kernel_time* out, int max_entries) {
 // Prefill workspace: [0, 256) device status word, then the path's scratch.
 static constexpr size_t kStatusBytes = 256;
 
+// ssd_debug_force_fma_prefill: every prefill takes the fp32-FMA path
+static std::atomic<int> g_force_fma{0};
+static bool use_tc(int P, int N, int io) { return prefill_tc_supported(P, N, io) && !g_force_fma.load(); }
+
 static size_t prefill_ws_bytes(int b, int T, int H, int P, int N, int chunk, int io) {
-    if (prefill_tc_supported(P, N, io)) return kStatusBytes + prefill_tc_workspace_bytes(b, T, H);
+    if (use_tc(P, N, io)) return kStatusBytes + prefill_tc_workspace_bytes(b, T, H);
     return kStatusBytes + prefill_simt_workspace_bytes(b, T, H, N, chunk, io);
 }
 
@@ -245,13 +249,13 @@ int ssd_debug_starve_next_prefill(unsigned long long wait_limit_ns) {
 
 int ssd_prefill_segments(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype) {
     if (check_prefill_shape(b, T, H, P, N, G, chunk, io_dtype) != SSD_OK) return 0;
-    if (b == 0 || T == 0 || !prefill_tc_supported(P, N, io_dtype)) return 1;
+    if (b == 0 || T == 0 || !use_tc(P, N, io_dtype)) return 1;
     return prefill_tc_segments(b, T, H);
 }
 
 int ssd_prefill_whole_units(int b, int T, int H, int P, int N, int G, int chunk, int io_dtype) {
     if (check_prefill_shape(b, T, H, P, N, G, chunk, io_dtype) != SSD_OK) return -1;
-    if (b == 0 || T == 0 || !prefill_tc_supported(P, N, io_dtype)) return b * H;
+    if (b == 0 || T == 0 || !use_tc(P, N, io_dtype)) return b * H;
     return prefill_tc_whole_units(b, T, H);
 }
 
@@ -337,6 +341,13 @@ int ssd_debug_force_prefill_split(int n_full, int nseg) {
     return SSD_OK;
 }
 
+int ssd_debug_force_fma_prefill(int on) {
+    g_detail[0] = 0;
+    if (on != 0 && on != 1) return set_error(SSD_ERR_INVALID_ARG, "on is %d, not 0 or 1", on);
+    g_force_fma.store(on);
+    return SSD_OK;
+}
+
 int ssd_debug_force_prefill_segments(int nseg) {
     g_detail[0] = 0;
     if (nseg < 0) return set_error(SSD_ERR_INVALID_ARG, "nseg %d is negative", nseg);
@@ -395,7 +406,7 @@ static int prefill_impl(int b, int T, int H, int P, int N, int G, int chunk, int
     if (overlaps({workspace, need}, ry)) return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps y");
     for (int i = 0; i < 7; ++i)
         if (overlaps({workspace, need}, rin[i])) return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps %s", names[i]);
-    if (prefill_tc_supported(P, N, io_dtype))
+    if (use_tc(P, N, io_dtype))
         return launch_prefill_tc(b, T, H, G, x, dt, dtm, A, B, C, D, h0, y, h_final, workspace, s);
     SSD_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(int), s));
     return launch_prefill_simt(b, T, H, N, G, chunk, io_dtype, x, dt, dtm, A, B, C, D, h0, y, h_final,

@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.ssd_debug_force_prefill_split.restype = _i
         L.ssd_debug_force_prefill_segments.argtypes = [_i]
         L.ssd_debug_force_prefill_segments.restype = _i
+        L.ssd_debug_force_fma_prefill.argtypes = [_i]
+        L.ssd_debug_force_fma_prefill.restype = _i
         L.ssd_decode_workspace_size.argtypes = [_i] * 3
         L.ssd_decode_workspace_size.restype = _sz
         L.ssd_decode_step.argtypes = [_i] * 9 + [_vp] * 10 + [_sz, _vp]
@@ -290,6 +292,12 @@ def debug_force_prefill_split(n_full, nseg):
     """Test hook: the first n_full (sequence, head) units run whole, the rest are split into
     nseg segments (nseg = 0: the cost model)."""
     _check(lib().ssd_debug_force_prefill_split(int(n_full), int(nseg)), "ssd_debug_force_prefill_split")
+
+
+def debug_force_fma_prefill(on=False):
+    """Measurement hook: route every following prefill through the fp32-FMA path, which uses
+    the chunk length as given (the tensor-core kernel always evaluates 128-token chunks)."""
+    _check(lib().ssd_debug_force_fma_prefill(1 if on else 0), "ssd_debug_force_fma_prefill")
 
 
 def debug_force_prefill_segments(nseg=0):

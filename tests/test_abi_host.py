@@ -195,6 +195,25 @@ def test_segment_hook_and_workspace():
         ssd.debug_force_prefill_segments(0)
 
 
+def test_fma_prefill_hook_routes_tensor_core_shapes_to_the_literal_chunk_path():
+    """With the hook on, a tensor-core shape is sized (and run) by the fp32-FMA path, whose
+    workspace depends on the chunk length; off, the tensor-core sizing ignores it."""
+    L = ssd.lib()
+    assert L.ssd_debug_force_fma_prefill(2) == INVALID and L.ssd_debug_force_fma_prefill(-1) == INVALID
+    shape = (2, 1024, 8, 64, 128, 1)
+    tc = {c: ssd.prefill_workspace_size(*shape, c, ssd.SSD_BF16) for c in (64, 128, 256)}
+    assert len(set(tc.values())) == 1
+    try:
+        ssd.debug_force_fma_prefill(True)
+        fma = {c: ssd.prefill_workspace_size(*shape, c, ssd.SSD_BF16) for c in (64, 128, 256)}
+        assert len(set(fma.values())) == 3
+        assert ssd.prefill_segments(*shape, 256, ssd.SSD_BF16) == 1
+        assert ssd.prefill_whole_units(*shape, 256, ssd.SSD_BF16) == 2 * 8
+    finally:
+        ssd.debug_force_fma_prefill(False)
+    assert ssd.prefill_workspace_size(*shape, 64, ssd.SSD_BF16) == tc[64]
+
+
 def test_decay_precision_hook_rejects_unknown_modes():
     L = ssd.lib()
     assert L.ssd_debug_decay_precision(3) == INVALID and L.ssd_debug_decay_precision(-1) == INVALID

@@ -228,6 +228,24 @@ def test_literal_chunk_length_vs_oracle(dtype, N, L):
     _full_check(case, chunk=L)
 
 
+@pytest.mark.parametrize("L", [64, 128, 256])
+def test_literal_chunk_length_at_tensor_core_shapes(L):
+    """ssd_debug_force_fma_prefill routes a tensor-core shape (bf16, N = 128, G = 8 as at
+    the long-context shape) through the fp32-FMA path, which uses the chunk length as given:
+    every L against the oracle, with a ragged last chunk.  This is the path the literal
+    chunk-length sweep is timed on."""
+    case = make_prefill(1, 3 * L + 37, 16, 64, 128, 8, L, "bf16", h0_std=0.1, seed=40 + L)
+    ssd.debug_force_fma_prefill(True)
+    try:
+        assert ssd.prefill_segments(case.b, case.T, case.H, 64, 128, 8, L, ssd.SSD_BF16) == 1
+        ssd.profile_begin()
+        _full_check(case, chunk=L)
+        kt = ssd.profile_end()
+    finally:
+        ssd.debug_force_fma_prefill(False)
+    assert "simt_chunk_output" in kt and "ssd_prefill_fused" not in kt
+
+
 # ------------------------------------------------------------------ edge cases
 def test_empty_sequence_passes_state_through():
     case = make_prefill(2, 256, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=10)
