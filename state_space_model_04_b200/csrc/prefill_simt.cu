@@ -64,23 +64,30 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int kPending>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
 
-// Copies a rows x W tile (row r at src_row(r), W contiguous elements; rows with !ok(r) are
-// zeros) into float shared memory, element (r, c) at dst[r * ld + c] or, transposed, at
+// Copies a kRows x W tile (row r at src + r * stride, W contiguous elements; rows r >= valid
+// are zeros) into float shared memory, element (r, c) at dst[r * ld + c] or, transposed, at
 // dst[c * ld + r]: asynchronously for fp32 inputs, through registers (converting) for bf16.
-template <int W, int kRows, bool kTransposed, typename RowPtr, typename RowOk>
-__device__ __forceinline__ void tile_load(float* dst, int ld, RowPtr src_row, RowOk ok) {
-    using IoT = typename std::remove_cv<typename std::remove_pointer<decltype(src_row(0))>::type>::type;
-    static_assert(kRows * W % kThreads == 0, "tile size");
+// A thread keeps one column c and walks rows kThreads / W apart, so each element costs one
+// pointer step.
+template <int W, int kRows, bool kTransposed, typename IoT>
+__device__ __forceinline__ void tile_load(float* dst, int ld, const IoT* src, size_t stride, int valid) {
+    static_assert(kThreads % W == 0 && kRows * W % kThreads == 0, "tile size");
+    constexpr int kStep = kThreads / W;  // rows between a thread's elements
+    const int c = threadIdx.x % W, r0 = threadIdx.x / W;
+    const IoT* s = src + r0 * stride + c;
+    const size_t s_step = kStep * stride;
+    float* d = kTransposed ? dst + c * ld + r0 : dst + r0 * ld + c;
+    const int d_step = kTransposed ? kStep : kStep * ld;
 #pragma unroll
-    for (int k = 0; k < kRows * W / kThreads; ++k) {
-        const int e = threadIdx.x + k * kThreads, r = e / W, c = e % W;
-        const bool v = ok(r);
-        float* d = kTransposed ? dst + c * ld + r : dst + r * ld + c;
+    for (int k = 0; k < kRows / kStep; ++k) {
+        const bool v = r0 + k * kStep < valid;
         if constexpr (std::is_same<IoT, float>::value) {
-            cp_async4(d, v ? src_row(r) + c : src_row(0), v);
+            cp_async4(d, v ? s : src, v);
         } else {
-            *d = v ? load_io(src_row(r), c) : 0.f;
+            *d = v ? load_io(s, 0) : 0.f;
         }
+        s += s_step;
+        d += d_step;
     }
 }
 
@@ -113,15 +120,22 @@ chunk_state_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __rest
     constexpr int XR = KT * kP / kThreads, BR = KT * N / kThreads;
     float xr[XR], br[BR];
     auto load_stage = [&](int k0) {
+        // thread column c (fixed), rows tid / W + k * (kThreads / W): one pointer step each
+        {
+            const int c = threadIdx.x % kP, r0 = threadIdx.x / kP;
+            const IoT* src = x + (((size_t)bi * T + t0 + k0 + r0) * H + hd) * kP + c;
+            const size_t step = (size_t)(kThreads / kP) * H * kP;
 #pragma unroll
-        for (int k = 0; k < XR; ++k) {
-            const int e = threadIdx.x + k * kThreads, t = k0 + e / kP;
-            xr[k] = t < Lc ? load_io(x, (((size_t)bi * T + t0 + t) * H + hd) * kP + e % kP) : 0.f;
+            for (int k = 0; k < XR; ++k, src += step)
+                xr[k] = k0 + r0 + k * (kThreads / kP) < Lc ? load_io(src, 0) : 0.f;
         }
+        {
+            const int c = threadIdx.x % N, r0 = threadIdx.x / N;
+            const IoT* src = Bm + (((size_t)bi * T + t0 + k0 + r0) * G + g) * N + c;
+            const size_t step = (size_t)(kThreads / N) * G * N;
 #pragma unroll
-        for (int k = 0; k < BR; ++k) {
-            const int e = threadIdx.x + k * kThreads, t = k0 + e / N;
-            br[k] = t < Lc ? load_io(Bm, (((size_t)bi * T + t0 + t) * G + g) * N + e % N) : 0.f;
+            for (int k = 0; k < BR; ++k, src += step)
+                br[k] = k0 + r0 + k * (kThreads / N) < Lc ? load_io(src, 0) : 0.f;
         }
     };
     load_stage(sl * KT);
@@ -407,11 +421,10 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
     auto issue_tile = [&](int t) {  // B, x, dt and the prefix sums of column tile t into slot t % kDepth
         if (t >= ntile) return;
         const int j0 = t * TJ, buf = t % kDepth;
-        auto ok = [&](int j) { return j0 + j < Lc; };
-        tile_load<N, TJ, true>(sBT + buf * N * kLdT, kLdT,
-                               [&](int j) { return Bm + (((size_t)bi * T + t0 + j0 + j) * G + g) * N; }, ok);
-        tile_load<kP, TJ, false>(sX + buf * TJ * kP, kP,
-                                 [&](int j) { return x + (((size_t)bi * T + t0 + j0 + j) * H + hd) * kP; }, ok);
+        tile_load<N, TJ, true>(sBT + buf * N * kLdT, kLdT, Bm + (((size_t)bi * T + t0 + j0) * G + g) * N,
+                               (size_t)G * N, Lc - j0);
+        tile_load<kP, TJ, false>(sX + buf * TJ * kP, kP, x + (((size_t)bi * T + t0 + j0) * H + hd) * kP,
+                                 (size_t)H * kP, Lc - j0);
         if (threadIdx.x < TJ) {
             const int j = j0 + threadIdx.x;
             s_dtj[buf][threadIdx.x] = j < Lc ? dt_value(dt[((size_t)bi * T + t0 + j) * H + hd], dtm, hd) : 0.f;
@@ -422,12 +435,11 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
     // copy groups, oldest first: {C, tile 0}, {H_in}, {tile 1} .. {tile kDepth - 1}, then one
     // per loop iteration (empty where there is no tile), so that tile t is complete once at
     // most kDepth - 1 groups are pending
-    tile_load<N, TR, false>(sC, LD, [&](int i) { return Cm + (((size_t)bi * T + t0 + i0 + i) * G + g) * N; },
-                            [&](int i) { return i0 + i < Lc; });
+    tile_load<N, TR, false>(sC, LD, Cm + (((size_t)bi * T + t0 + i0) * G + g) * N, (size_t)G * N, Lc - i0);
     issue_tile(0);
     cp_async_commit();
     const float* Hc = Hin + (((size_t)bi * nc + c) * H + hd) * ks * kP * N;
-    tile_load<N, kP, true>(sHT, kLdT, [&](int p) { return Hc + (size_t)p * N; }, [](int) { return true; });
+    tile_load<N, kP, true>(sHT, kLdT, Hc, (size_t)N, kP);
     cp_async_commit();
 #pragma unroll
     for (int t = 1; t < kDepth; ++t) {
