@@ -610,7 +610,7 @@ def decay_precision_ablation(ssd, torch, dev):
 
 def bench_prefill_configs(ssd, torch, dev, stream, args, clocks, barrier, max_over_ranks, world, pk, box):
     """The other prefill configurations: the tiny fp32 case (b=1, T=512, H=4, N=64; the fp32
-    four-kernel path, launch-latency bound), the 130M-layer shape (b=1, T=4096, H=24) and the
+    three-kernel fp32-FMA path, launch-latency bound), the 130M-layer shape (b=1, T=4096, H=24) and the
     long-context shape (b=1, T=65536, H=80, G=8), inputs resident in HBM, each step timed
     alone with CUDA events on the launching stream after a write that evicts L2, max over
     ranks; the per-kernel times come from a second pass with events around every launch.  The fused tensor-core path

@@ -90,13 +90,14 @@ SSD_API const char* ssd_last_error(void);
  * chunk must be 64, 128 or 256.  x, B, C, dt, A, D must not alias y or h_final.
  * Arithmetic: SSD_BF16 inputs with P == 64 and N == 128 run one fused tensor-core kernel
  * (tcgen05 bf16 contractions, fp32 accumulation, fp32 decay in log space, fp32 running
- * state kept on chip), after a tensor-core state pass and a scan when few (sequence,
- * head) pairs would leave SMs idle (sequences split into segments, see
- * ssd_prefill_segments).  THAT KERNEL IGNORES `chunk`: it always evaluates the chunked
+ * state kept on chip), after a tensor-core state pass when (sequence, head) pairs would
+ * leave SMs idle (some or all sequences split into segments whose entering states the
+ * fused kernel folds from the state pass's results; see ssd_prefill_segments and
+ * ssd_prefill_whole_units).  THAT KERNEL IGNORES `chunk`: it always evaluates the chunked
  * form with 128-token chunks (one tcgen05 tile of rows), whatever chunk length is passed
  * (64, 128 or 256 are accepted and give bitwise the same result).  Every chunk length
  * computes the same function; only the rounding and the operation count differ.  Other
- * bf16 shapes and all SSD_F32 inputs run the four-kernel fp32-FMA path, which uses
+ * bf16 shapes and all SSD_F32 inputs run the three-kernel fp32-FMA path, which uses
  * `chunk` as given, with the prefix sums of dt*A kept in fp64 (no TF32).
  * The workspace's first 256 bytes hold a device status word (see ssd_prefill_check).
  * Errors: SSD_ERR_INVALID_ARG (null pointer for a required argument, negative size,

@@ -1001,7 +1001,9 @@ ssd_prefill_fused_kernel(const __grid_constant__ TcParams prm) {
 // ------------------------------------------------------------------ segment state pass
 // For a sequence split into segments, the state a segment leaves behind when it starts
 // from zero ("Chunked recurrence" run over the segment alone) and the segment's total log
-// decay sum(dt*A).  A scan over segments then gives every segment its entering state.
+// decay sum(dt*A); the first segment's end state starts from h0.  Folding the earlier
+// segments' end states in order gives every later segment its entering state (the fused
+// kernel does that itself, or the prefix pass below when there are many segments).
 // One CTA per segment of kHP heads of one sequence that share a B/C group: with kHP = 2 the
 // group's B tile is loaded once for both heads and one MMA (N = 128) serves both, which cuts
 // the bytes a block moves from 48 KB per head to 32 KB.

@@ -222,7 +222,7 @@ def test_tensor_core_path_ignores_chunk():
 @pytest.mark.parametrize("L", [64, 128, 256])
 @pytest.mark.parametrize("dtype,N", [("f32", 64), ("bf16", 64)])
 def test_literal_chunk_length_vs_oracle(dtype, N, L):
-    """The four-kernel path (fp32 inputs, or N = 64) evaluates the chunked form with the
+    """The fp32-FMA path (fp32 inputs, or N = 64) evaluates the chunked form with the
     chunk length given: every L against the oracle, with a ragged last chunk."""
     case = make_prefill(1, 3 * L + 37, 4, 64, N, 2, L, dtype, h0_std=0.1, seed=10 + L)
     _full_check(case, chunk=L)
@@ -340,7 +340,7 @@ def _raw_dt(b, T, H, seed):
 @pytest.mark.parametrize("dtype,shape,nseg", [
     ("bf16", (2, 700, 6, 64, 128, 3), 1),     # fused tensor-core pass
     ("bf16", (2, 700, 6, 64, 128, 3), 3),     # segment state pass + scan + fused pass
-    ("bf16", (1, 300, 4, 64, 64, 2), 0),      # N = 64: the four-kernel path
+    ("bf16", (1, 300, 4, 64, 64, 2), 0),      # N = 64: the fp32-FMA path
     ("f32", (1, 512, 4, 64, 64, 1), 0),       # fp32 gate
 ])
 def test_dt_raw_matches_oracle(dtype, shape, nseg):

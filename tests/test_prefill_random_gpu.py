@@ -5,7 +5,7 @@ against every block and chunk length), 2-8 heads in 1-H groups, N = 64 or 128, b
 fp32, chunk 64/128/256, a forced segment count (automatic, 1, 2 or 5) and a zero or random
 initial state, and compares y and h_final with the oracle within the dtype's bound.  The
 draws cover the fused tensor-core path (bf16, N = 128) with and without sequence splits,
-and the four-kernel path (fp32 or N = 64).
+and the fp32-FMA path (fp32 or N = 64).
 """
 import numpy as np
 import pytest
