@@ -326,6 +326,41 @@ def test_in_place_state_resume(nseg):
     assert torch.equal(y2, y) and torch.equal(h, hf)
 
 
+def test_back_to_back_chained_calls_match_single_calls():
+    """Split prefills issued back to back on one stream and one workspace, alternating two
+    inputs and in-place state updates, with no host synchronisation between them: the
+    chained grids (status reset, state pass, fused pass, each allowed to start before the
+    one ahead ends) give bitwise what one synchronised call each gives."""
+    cases = [make_prefill(2, 1000, 6, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=s) for s in (71, 72)]
+    ins = [prefill_inputs(c) for c in cases]
+    ssd.debug_force_prefill_segments(4)
+    try:
+        ws = torch.empty(ssd.prefill_workspace_size(2, 1000, 6, 64, 128, 1, 256, ssd.SSD_BF16),
+                         dtype=torch.uint8, device="cuda")
+        # reference: each call alone, synchronised; the state of each input chained 3 times
+        ref = []
+        for t in ins:
+            h = t["h0"].clone()
+            for _ in range(3):
+                y, _ = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=256, h0=h, h_final=h,
+                                   workspace=ws)
+                torch.cuda.synchronize()
+            ref.append((y.clone(), h.clone()))
+        # the same calls interleaved, no synchronisation until the end
+        hs = [t["h0"].clone() for t in ins]
+        ys = [torch.empty_like(t["x"]) for t in ins]
+        for _ in range(3):
+            for i, t in enumerate(ins):
+                ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=256, h0=hs[i], h_final=hs[i],
+                            y=ys[i], workspace=ws, check=False)
+        torch.cuda.synchronize()
+        ssd.prefill_check(ws)
+    finally:
+        ssd.debug_force_prefill_segments(0)
+    for i in range(2):
+        assert torch.equal(ys[i], ref[i][0]) and torch.equal(hs[i], ref[i][1])
+
+
 # ------------------------------------------------------------------ raw dt pre-processing
 def _raw_dt(b, T, H, seed):
     """Raw steps whose softplus follows the input recipe: bias = softplus^-1 of a log-uniform
