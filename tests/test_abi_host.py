@@ -214,6 +214,25 @@ def test_fma_prefill_hook_routes_tensor_core_shapes_to_the_literal_chunk_path():
     assert ssd.prefill_workspace_size(*shape, 64, ssd.SSD_BF16) == tc[64]
 
 
+def test_split_planner_decisions_on_148_sms():
+    """The split planner's choices at the configurations' shapes (148 SMs, the count used
+    when no device is visible): the 130M-layer shape in 6 segments, the long-context shape
+    in 11, the 2.7B-layer shape with the 48 pairs of its ragged last wave in 3 segments, and
+    a shape whose pairs fill whole waves unsplit."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("decisions depend on the device's SM count")
+    bf16 = ssd.SSD_BF16
+    assert ssd.prefill_segments(1, 4096, 24, 64, 128, 1, 256, bf16) == 6
+    assert ssd.prefill_whole_units(1, 4096, 24, 64, 128, 1, 256, bf16) == 0
+    assert ssd.prefill_segments(1, 65536, 80, 64, 128, 8, 256, bf16) == 11
+    assert ssd.prefill_whole_units(1, 65536, 80, 64, 128, 8, 256, bf16) == 0
+    assert ssd.prefill_segments(8, 4096, 80, 64, 128, 1, 256, bf16) == 3
+    assert ssd.prefill_whole_units(8, 4096, 80, 64, 128, 1, 256, bf16) == 592
+    assert ssd.prefill_segments(74, 4096, 4, 64, 128, 1, 256, bf16) == 1   # 296 pairs: two whole waves
+    assert ssd.prefill_whole_units(74, 4096, 4, 64, 128, 1, 256, bf16) == 296
+
+
 def test_decay_precision_hook_rejects_unknown_modes():
     L = ssd.lib()
     assert L.ssd_debug_decay_precision(3) == INVALID and L.ssd_debug_decay_precision(-1) == INVALID
