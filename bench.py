@@ -7,8 +7,8 @@ Workload (per rank; ranks process independent batches, so scaling is weak):
   * prefill, the headline: the 2.7B-layer shape -- b=8 sequences x T=4096 tokens,
     H=80 heads, P=64, N=128, G=1, chunk 256, bf16 x/B/C, fp32 dt/A/D, h0 ~ N(0, 0.1).
     One step = one ssd_prefill call over that batch.  value = TFLOP/s of the chunked
-    decomposition that ran (128-token chunks on the fused tensor-core path), with the
-    L = 256 count beside it; tokens/s does not depend on the decomposition.
+    decomposition that ran (128-token chunks on the fused tensor-core path,
+    chunk_executed); tokens/s does not depend on the decomposition.
   * cached decode at the 2.7B shape: 64 layers x (80 x 64 x 128) fp32 state + width-4
     conv over 5376 channels, batch 1 (and 32), state from the prefill's final state,
     run as graph launches of on-device steps; reported under "decode".
@@ -16,7 +16,8 @@ Inputs are seeded synthetic draws (ssd_inputs); the per-step prefill inputs (740
 exceed the 126 MB L2, so no flush is needed between steps.
 
 Prints ONE JSON line on rank 0.  gpu_launches counts our kernel launches inside the timed
-region that `value` measures (two per step: the status reset and the fused prefill);
+region that `value` measures (three per step at the headline shape: the status reset, the
+segment state pass for the pairs of the ragged last wave, the fused prefill);
 gpu_launches_all_timed_regions adds those of the per-kernel timing, decode, raw-dt and
 other-configuration regions.  --impl reference times the CPU oracle (the only
 reference this method has: an fp64 C implementation of the recurrence) on bounded
