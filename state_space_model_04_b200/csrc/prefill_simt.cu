@@ -570,6 +570,8 @@ int run(int b, int T, int H, int G, int L, const void* x, const float* dt, const
     const IoT* xi = static_cast<const IoT*>(x);
     const IoT* Bi = static_cast<const IoT*>(Bm);
     const IoT* Ci = static_cast<const IoT*>(Cm);
+    if (const int st = smem_limit_once((const void*)chunk_state_kernel<IoT, CsT, N>, 0)) return st;
+    if (const int st = smem_limit_once((const void*)state_scan_kernel<CsT, N>, 0)) return st;
     {
         LaunchScope ls("simt_chunk_state", s);
         chunk_state_kernel<IoT, CsT, N><<<dim3(nc * ks, H, b), kThreads, 0, s>>>(T, H, G, L, nc, ks, xi, dt, dtm, A, Bi,

@@ -1263,6 +1263,7 @@ cudaError_t launch_pdl(void (*k)(Param), unsigned grid, unsigned block, size_t s
 }
 
 int reset_status(int* status, cudaStream_t s) {
+    if (const int st = smem_limit_once((const void*)ssd_status_reset_kernel, 0)) return st;
     {
         LaunchScope ls("ssd_status_reset", s);
         ssd_status_reset_kernel<<<1, 32, 0, s>>>(status);
@@ -1601,6 +1602,7 @@ int launch_prefill_tc(int b, int T, int H, int G, const void* x, const float* dt
     if ((st = reset_status(prm.status, s)) != SSD_OK) return st;
     if (prm.nseg > 1 && (st = launch_state_pass(prm, n_split, decay, s)) != SSD_OK) return st;
     if (prm.seg_prefix) {
+        if ((st = smem_limit_once((const void*)ssd_segment_prefix_kernel, 0)) != SSD_OK) return st;
         LaunchScope ls("ssd_segment_prefix", s);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)n_split, 1, kScanSplit);
