@@ -143,6 +143,37 @@ def test_scalar_impulse_response():
     np.testing.assert_allclose(y.reshape(-1), d * np.exp(d * Av * t), rtol=1e-13)
 
 
+@pytest.mark.parametrize("form", ["recurrence", "chunked8", "chunked16", "quadratic"])
+def test_step_response_closed_form(form):
+    """Constant x, B, C, dt and A with a nonzero h0: the recurrence is a geometric series,
+    h_t = q^(t+1) h0 + dt x B^T (1 - q^(t+1)) / (1 - q) with q = exp(dt*A), and
+    y_t = h_t C + D x.  T = 48 spans six chunks of 8 and three of 16 (the oracle's chunked
+    form takes whole chunks), so a dropped or mis-indexed inter-chunk term, or the initial
+    state applied at the wrong token, moves y away from the series."""
+    T, P, N, d, Av, Dv = 48, 2, 3, 0.21, -0.8, 0.5
+    xv = np.array([0.7, -1.1])
+    bv = np.array([0.4, -0.3, 1.2])
+    cv = np.array([-0.6, 0.9, 0.25])
+    h0v = np.array([[0.3, -0.2, 0.1], [0.05, 0.4, -0.35]])
+    x = np.broadcast_to(xv, (1, T, 1, P)).copy()
+    dt = np.full((1, T, 1), d)
+    Bm = np.broadcast_to(bv, (1, T, 1, N)).copy()
+    Cm = np.broadcast_to(cv, (1, T, 1, N)).copy()
+    h0 = h0v.reshape(1, 1, P, N)
+    args = (x, dt, np.array([Av]), Bm, Cm, np.array([Dv]))
+    if form == "recurrence":
+        y, hf = oracle.ssd_recurrence(*args, h0)
+    elif form == "quadratic":
+        y, hf = oracle.ssd_quadratic(*args, h0)
+    else:
+        y, hf = oracle.ssd_chunked(*args, int(form[len("chunked"):]), h0)
+    q = np.exp(d * Av)
+    n = np.arange(1, T + 1)[:, None, None]                       # tokens folded in after h0
+    h = q ** n * h0v + d * np.outer(xv, bv) * (1 - q ** n) / (1 - q)   # [T, P, N]
+    np.testing.assert_allclose(y.reshape(T, P), h @ cv + Dv * xv, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(hf.reshape(P, N), h[-1], rtol=1e-12, atol=1e-14)
+
+
 # ---------------------------------------------------------------- invariants
 def test_split_resume():
     """prefill(T1+T2, h0) == prefill(T2, h_final(prefill(T1, h0))): the cache hand-off."""
