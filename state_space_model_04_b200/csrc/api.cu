@@ -81,8 +81,8 @@ int smem_limit_once(const void* func, int bytes) {
         if (std::get<0>(d) == func && std::get<1>(d) == dev && std::get<2>(d) >= bytes) return SSD_OK;
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(MaxDynamicSharedMemorySize)");
-    // every kernel of the library asks for the largest shared-memory carveout, so that small
-    // kernels launched between large ones leave the SMs' L1/shared split as it is
+    // the single-GPU prefill kernels all ask for the largest shared-memory carveout, so that
+    // the small ones launched between large ones leave the SMs' L1/shared split as it is
     e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return cuda_status(e, "cudaFuncSetAttribute(PreferredSharedMemoryCarveout)");
     done.emplace_back(func, dev, bytes);
