@@ -15,8 +15,11 @@
 //   K4 chunk_output   y_i = sum_{j<=i} (C_i.B_j) exp(cs_i-cs_j) dt_j x_j
 //                           + exp(cs_i) C_i.H_c + D x_i
 // When (chunks x heads x sequences) alone would leave most SMs idle, the chunk state is
-// split over slices of 32 tokens and the output over 16-row tiles; the partial states are
-// added in a fixed order, so results stay bitwise reproducible.
+// split over slices of 32 tokens and the output over 16-row tiles whose products are split
+// into four quarters of their contraction; partial states and quarters are added in a fixed
+// order, so results are bitwise reproducible from run to run.  The two output kernels sum in
+// different orders, so a batch size that moves a call from one to the other changes y by
+// rounding only.
 //
 // This path serves fp32 inputs: every product and sum is an fp32 FMA (no TF32), and the
 // prefix sums are kept in fp64 (CsT = double) so that exp(cs_i - cs_j) keeps full fp32
@@ -375,21 +378,37 @@ chunk_output_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __res
 }
 
 // K4 for grids too small to fill the GPU: one CTA = 16 output rows of one chunk of one
-// (sequence, head); thread (row, group of four columns).  B and H_in are kept transposed
-// ([n][j], [n][p]) and x row-major, so that every step of the three products reads the
-// thread's four columns with one 16-byte shared load beside one broadcast value (these
-// small grids are bound by shared-memory issue, not by arithmetic).  All copies are
-// asynchronous into a ring of kDepth column tiles (the whole 256-token chunk at N = 64), so
-// up to kDepth - 1 tiles are in flight while one is evaluated.  Same arithmetic, in the same
-// order, as chunk_output_kernel.
-constexpr int kSmallRows = 16, kSmallCols = 64, kLdT = 68;  // transposed rows: 64 + 4 (16-byte aligned)
+// (sequence, head).  The CTAs of rows late in a chunk see up to four 64-column tiles and set
+// the kernel's length, so each product is register-blocked to shorten their serial chain: a
+// thread owns a 4 x 4 block of its output and one quarter of the contraction (kq =
+// threadIdx.x / 64), and one step reads two 16-byte shared values (four rows of one operand,
+// four columns of the other) for sixteen FMAs.  The quarters are added in order through
+// shared memory: the scores after every column tile, y once at the end.  C, B and H_in are
+// kept transposed ([n][i], [n][j], [n][p]), the masked decayed scores transposed ([j][i]),
+// x row-major.  All copies are asynchronous into a ring of kDepth column tiles (the whole
+// 256-token chunk at N = 64), so up to kDepth - 1 tiles are in flight while one is evaluated.
+constexpr int kSmallRows = 16, kSmallCols = 64;
+constexpr int kLdT = 68, kLdR = 20;  // rows of 64 and of 16 floats, padded to keep 16-byte alignment
+constexpr int kSplit = kThreads / ((kSmallRows / 4) * (kSmallCols / 4));  // contraction quarters
 template <int N>
 constexpr int small_depth() { return N == 64 ? 4 : 2; }
 template <int N>
 constexpr size_t small_smem_bytes() {
-    return sizeof(float) * (kSmallRows * (N + 1) + N * kLdT + small_depth<N>() * (N * kLdT + kSmallCols * kP) +
-                            kSmallRows * (kSmallCols + 1));
+    return sizeof(float) * (N * kLdR + N * kLdT + small_depth<N>() * (N * kLdT + kSmallCols * kP) +
+                            kSplit * kSmallRows * kLdT + kSmallCols * kLdR);
 }
+
+// a[r][q] += u[r] * v[q]
+__device__ __forceinline__ void fma_4x4(float (&a)[4][4], const float4 u, const float4 v) {
+    const float ur[4] = {u.x, u.y, u.z, u.w}, vq[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a[r][q] = fmaf(ur[r], vq[q], a[r][q]);
+}
+
+__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
 template <typename IoT, typename CsT, int N>
 __global__ void __launch_bounds__(kThreads)
 chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT* __restrict__ x,
@@ -397,14 +416,16 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
                           const IoT* __restrict__ Cm, const float* __restrict__ D,
                           const CsT* __restrict__ cs, const float* __restrict__ Hin,
                           IoT* __restrict__ y) {
-    constexpr int TR = kSmallRows, TJ = kSmallCols, LD = N + 1, kDepth = small_depth<N>();
-    static_assert(TJ == kP && TR * 16 == kThreads, "thread (row, four columns of j and of p)");
+    constexpr int TR = kSmallRows, TJ = kSmallCols, kDepth = small_depth<N>();
+    constexpr int NQ = N / kSplit, JQ = TJ / kSplit;  // contraction length of one quarter
+    static_assert(TJ == kP && kSplit == 4 && TR * TJ == 4 * kThreads, "4 x 4 blocks, four quarters");
     extern __shared__ __align__(16) float smem[];
-    float* sC = smem;                     // [TR][LD]            C rows i
-    float* sHT = sC + TR * LD;            // [N][kLdT]           H_in, transposed: [n][p]
-    float* sBT = sHT + N * kLdT;          // [kDepth][N][kLdT]   B, transposed: [n][j]
-    float* sX = sBT + kDepth * N * kLdT;  // [kDepth][TJ][kP]    x rows j
-    float* sG = sX + kDepth * TJ * kP;    // [TR][TJ + 1]        masked decayed C.B^T
+    float* sCT = smem;                     // [N][kLdR]            C, transposed: [n][i]
+    float* sHT = sCT + N * kLdR;           // [N][kLdT]            H_in, transposed: [n][p]
+    float* sBT = sHT + N * kLdT;           // [kDepth][N][kLdT]    B, transposed: [n][j]
+    float* sX = sBT + kDepth * N * kLdT;   // [kDepth][TJ][kP]     x rows j
+    float* sQ = sX + kDepth * TJ * kP;     // [kSplit][TR][kLdT]   quarter partials: scores, then y
+    float* sGT = sQ + kSplit * TR * kLdT;  // [TJ][kLdR]           masked decayed scores, transposed: [j][i]
     __shared__ CsT s_csi[TR];
     __shared__ CsT s_csj[kDepth][TJ];
     __shared__ float s_dtj[kDepth][TJ];
@@ -416,7 +437,8 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
     if (i0 >= Lc) return;
     const int ntile = (min(i0 + TR, Lc) + TJ - 1) / TJ;  // column tiles at and below the diagonal
     const CsT* csc = cs + (((size_t)bi * H + hd) * nc + c) * L;
-    const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;  // row i0 + tr, columns 4 tc .. 4 tc + 3
+    // quarter kq of the contraction; output rows 4 ri .. 4 ri + 3, columns 4 ci .. 4 ci + 3
+    const int kq = threadIdx.x / 64, ri = (threadIdx.x % 64) / 16, ci = threadIdx.x % 16;
 
     auto issue_tile = [&](int t) {  // B, x, dt and the prefix sums of column tile t into slot t % kDepth
         if (t >= ntile) return;
@@ -435,7 +457,7 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
     // copy groups, oldest first: {C, tile 0}, {H_in}, {tile 1} .. {tile kDepth - 1}, then one
     // per loop iteration (empty where there is no tile), so that tile t is complete once at
     // most kDepth - 1 groups are pending
-    tile_load<N, TR, false>(sC, LD, Cm + (((size_t)bi * T + t0 + i0) * G + g) * N, (size_t)G * N, Lc - i0);
+    tile_load<N, TR, true>(sCT, kLdR, Cm + (((size_t)bi * T + t0 + i0) * G + g) * N, (size_t)G * N, Lc - i0);
     issue_tile(0);
     cp_async_commit();
     const float* Hc = Hin + (((size_t)bi * nc + c) * H + hd) * ks * kP * N;
@@ -450,21 +472,19 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
     cp_async_wait<kDepth - 1>();  // C, tile 0 and H_in landed
     __syncthreads();
 
-    // state-to-output term: Y[i][p] = exp(cs_i) * sum_n C[i][n] H[p][n]
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int n = 0; n < N; ++n) {
-        const float cv = sC[tr * LD + n];
-        const float4 h4 = *reinterpret_cast<const float4*>(sHT + n * kLdT + 4 * tc);
-        acc[0] = fmaf(cv, h4.x, acc[0]);
-        acc[1] = fmaf(cv, h4.y, acc[1]);
-        acc[2] = fmaf(cv, h4.z, acc[2]);
-        acc[3] = fmaf(cv, h4.w, acc[3]);
-    }
+    const float* cq = sCT + kq * NQ * kLdR + 4 * ri;  // this thread's C rows, from its quarter's first n
+    // state-to-output term, this quarter of n: Y[i][p] = exp(cs_i) * sum_n C[i][n] H[p][n]
+    float acc[4][4] = {};
     {
-        const float e = exp_cs(s_csi[tr]);
+        const float* hq = sHT + kq * NQ * kLdT + 4 * ci;
+#pragma unroll 4
+        for (int n = 0; n < NQ; ++n) fma_4x4(acc, lds4(cq + n * kLdR), lds4(hq + n * kLdT));
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc[q] *= e;
+        for (int r = 0; r < 4; ++r) {
+            const float e = exp_cs(s_csi[4 * ri + r]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[r][q] *= e;
+        }
     }
 
     // intra-chunk dual form over the column tiles
@@ -475,47 +495,70 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
             cp_async_wait<kDepth - 1>();  // tile t landed
             __syncthreads();
         }
-        const float* sBt = sBT + buf * N * kLdT;
-        const float* sXt = sX + buf * TJ * kP;
-        float gacc[4] = {0.f, 0.f, 0.f, 0.f};
+        {   // scores, this quarter of n: S[i][j] = sum_n C[i][n] B[j][n]
+            const float* bq = sBT + buf * N * kLdT + kq * NQ * kLdT + 4 * ci;
+            float sc[4][4] = {};
 #pragma unroll 4
-        for (int n = 0; n < N; ++n) {
-            const float cv = sC[tr * LD + n];
-            const float4 b4 = *reinterpret_cast<const float4*>(sBt + n * kLdT + 4 * tc);
-            gacc[0] = fmaf(cv, b4.x, gacc[0]);
-            gacc[1] = fmaf(cv, b4.y, gacc[1]);
-            gacc[2] = fmaf(cv, b4.z, gacc[2]);
-            gacc[3] = fmaf(cv, b4.w, gacc[3]);
-        }
+            for (int n = 0; n < NQ; ++n) fma_4x4(sc, lds4(cq + n * kLdR), lds4(bq + n * kLdT));
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int jl = 4 * tc + q;
-            float v = 0.f;
-            if (j0 + jl <= i0 + tr) v = gacc[q] * exp_cs(s_csi[tr] - s_csj[buf][jl]) * s_dtj[buf][jl];
-            sG[tr * (TJ + 1) + jl] = v;
+            for (int r = 0; r < 4; ++r)
+                *reinterpret_cast<float4*>(sQ + (kq * TR + 4 * ri + r) * kLdT + 4 * ci) =
+                    make_float4(sc[r][0], sc[r][1], sc[r][2], sc[r][3]);
         }
         __syncthreads();
-#pragma unroll 4
-        for (int j = 0; j < TJ; ++j) {
-            const float gv = sG[tr * (TJ + 1) + j];
-            const float4 x4 = *reinterpret_cast<const float4*>(sXt + j * kP + 4 * tc);
-            acc[0] = fmaf(gv, x4.x, acc[0]);
-            acc[1] = fmaf(gv, x4.y, acc[1]);
-            acc[2] = fmaf(gv, x4.z, acc[2]);
-            acc[3] = fmaf(gv, x4.w, acc[3]);
+        {   // the quarters added in order, then the decay and the causal mask: thread (column
+            // jl, rows 4 r4 .. 4 r4 + 3) writes one 16-byte row of the transposed scores
+            const int jl = threadIdx.x % TJ, r4 = threadIdx.x / TJ;
+            float v[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int i = 4 * r4 + r;
+                float sv = sQ[i * kLdT + jl];
+#pragma unroll
+                for (int q = 1; q < kSplit; ++q) sv += sQ[(q * TR + i) * kLdT + jl];
+                v[r] = j0 + jl <= i0 + i ? sv * exp_cs(s_csi[i] - s_csj[buf][jl]) * s_dtj[buf][jl] : 0.f;
+            }
+            *reinterpret_cast<float4*>(sGT + jl * kLdR + 4 * r4) = make_float4(v[0], v[1], v[2], v[3]);
         }
-        __syncthreads();  // slot t % kDepth and the score tile are free
+        __syncthreads();
+        // this quarter of the tile's columns: Y[i][p] += sum_j S~[i][j] x[j][p]; a quarter wholly
+        // above the diagonal adds nothing (kq is the same across a warp)
+        if (j0 + kq * JQ <= i0 + TR - 1) {
+            const float* gq = sGT + kq * JQ * kLdR + 4 * ri;
+            const float* xq = sX + buf * TJ * kP + kq * JQ * kP + 4 * ci;
+#pragma unroll 4
+            for (int j = 0; j < JQ; ++j) fma_4x4(acc, lds4(gq + j * kLdR), lds4(xq + j * kP));
+        }
+        __syncthreads();  // slot t % kDepth, the partials and the scores are free
         issue_tile(t + kDepth);
         cp_async_commit();
     }
-    const int i = i0 + tr;
+
+    // the quarters of y added in order, then the D skip: thread (row, columns 4 pc .. 4 pc + 3)
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+        *reinterpret_cast<float4*>(sQ + (kq * TR + 4 * ri + r) * kLdT + 4 * ci) =
+            make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+    __syncthreads();
+    const int row = threadIdx.x / 16, pc = threadIdx.x % 16;
+    const int i = i0 + row;
     if (i < Lc) {
+        float4 sv = lds4(sQ + row * kLdT + 4 * pc);
+#pragma unroll
+        for (int q = 1; q < kSplit; ++q) {
+            const float4 u = lds4(sQ + (q * TR + row) * kLdT + 4 * pc);
+            sv.x += u.x;
+            sv.y += u.y;
+            sv.z += u.z;
+            sv.w += u.w;
+        }
+        const float out[4] = {sv.x, sv.y, sv.z, sv.w};
         const float Dv = D[hd];
         const size_t off = (((size_t)bi * T + t0 + i) * H + hd) * kP;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int p = 4 * tc + q;
-            store_io(y, off + p, acc[q] + Dv * load_io(x, off + p));
+            const int p = 4 * pc + q;
+            store_io(y, off + p, out[q] + Dv * load_io(x, off + p));
         }
     }
 }
@@ -543,8 +586,8 @@ int state_slices(int b, int T, int H, int N, int L) {
     return ks;
 }
 
-// K4: 64-row tiles, or the pipelined 16-row kernel when 64-row tiles would not give every
-// SM two CTAs
+// K4: 64-row tiles, or the pipelined, register-blocked 16-row kernel when 64-row tiles would
+// not give every SM two CTAs
 template <typename IoT, typename CsT, int N>
 int launch_output(int b, int T, int H, int G, int L, int nc, int ks, const IoT* x, const float* dt, const DtMap& dtm,
                   const IoT* Bm, const IoT* Cm, const float* D, const CsT* cs, const float* S, void* y, cudaStream_t s) {
