@@ -99,6 +99,10 @@ SSD_API const char* ssd_last_error(void);
  * computes the same function; only the rounding and the operation count differ.  Other
  * bf16 shapes and all SSD_F32 inputs run the three-kernel fp32-FMA path, which uses
  * `chunk` as given, with the prefix sums of dt*A kept in fp64 (no TF32).
+ * Determinism: no floating-point atomics; the same call gives bitwise the same y and
+ * h_final every time.  A sequence's result can depend on the rest of the batch by rounding
+ * only: it is bitwise the same whenever the kernels and segment split chosen for the call
+ * are the same (both depend on b * H and, on the fp32 path, on the chunk count).
  * The workspace's first 256 bytes hold a device status word (see ssd_prefill_check).
  * Errors: SSD_ERR_INVALID_ARG (null pointer for a required argument, negative size,
  * H % G != 0, bad chunk or dtype, misaligned pointer), SSD_ERR_UNSUPPORTED (P, N),
