@@ -1507,7 +1507,9 @@ int prefill_tc_whole_units(int b, int T, int H) {
 }
 
 // Workspace: the status word, then (split sequences only) the segments' end states, their
-// log decays, and room for a copy of the split units' h0.
+// log decays, and room for a copy of h0 for when h0 and h_final are one buffer.  The fused
+// kernel reads that copy at the same unit offsets as h0, and the copy holds the split units
+// [n_full, b*H) only, so its room spans all b*H units.
 struct SplitLayout {
     size_t state, logdecay, h0copy, bytes;
 };
@@ -1517,7 +1519,7 @@ SplitLayout split_layout(int b, int H, const SplitPlan& sp) {
     l.state = kSegOffset;
     l.logdecay = l.state + align256(units * kP * kN * sizeof(float));
     l.h0copy = l.logdecay + align256(units * sizeof(float));
-    l.bytes = l.h0copy + align256(n_split * kP * kN * sizeof(float));
+    l.bytes = l.h0copy + align256((size_t)b * H * kP * kN * sizeof(float));
     return l;
 }
 

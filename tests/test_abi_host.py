@@ -233,6 +233,32 @@ def test_split_planner_decisions_on_148_sms():
     assert ssd.prefill_whole_units(74, 4096, 4, 64, 128, 1, 256, bf16) == 296
 
 
+def _split_workspace_floor(units, n_full, nseg, P=64, N=128):
+    """Bytes a split tensor-core prefill touches in its workspace: the 512-byte header, one
+    fp32 state and one log decay per split unit and segment but the last, and the in-place
+    copy of h0, which the fused kernel reads at the same unit offsets as h0 itself (units
+    n_full .. units - 1), so it reaches units * P * N floats past its start."""
+    seg = (units - n_full) * (nseg - 1)
+    return 512 + seg * P * N * 4 + seg * 4 + units * P * N * 4
+
+
+def test_workspace_holds_the_in_place_h0_copy_when_some_units_run_whole():
+    """h_final aliasing h0 with only the ragged last wave split (the 2.7B-layer shape: 592
+    pairs whole, 48 in 3 segments) and with a forced partial split: the workspace the query
+    returns covers the h0 copy at the split units' own offsets."""
+    bf16 = ssd.SSD_BF16
+    assert ssd.prefill_whole_units(8, 4096, 80, 64, 128, 1, 256, bf16) == 592
+    assert ssd.prefill_segments(8, 4096, 80, 64, 128, 1, 256, bf16) == 3
+    assert ssd.prefill_workspace_size(8, 4096, 80, 64, 128, 1, 256, bf16) >= _split_workspace_floor(640, 592, 3)
+    ssd.debug_force_prefill_split(100, 4)
+    try:
+        assert ssd.prefill_whole_units(2, 1024, 80, 64, 128, 1, 256, bf16) == 100
+        assert ssd.prefill_segments(2, 1024, 80, 64, 128, 1, 256, bf16) == 4
+        assert ssd.prefill_workspace_size(2, 1024, 80, 64, 128, 1, 256, bf16) >= _split_workspace_floor(160, 100, 4)
+    finally:
+        ssd.debug_force_prefill_split(0, 0)
+
+
 def test_decay_precision_hook_rejects_unknown_modes():
     L = ssd.lib()
     assert L.ssd_debug_decay_precision(3) == INVALID and L.ssd_debug_decay_precision(-1) == INVALID

@@ -326,6 +326,27 @@ def test_in_place_state_resume(nseg):
     assert torch.equal(y2, y) and torch.equal(h, hf)
 
 
+def test_in_place_state_resume_with_whole_units():
+    """h_final aliasing h0 when some units run whole and the rest are split (the kind of
+    plan the cost model picks for a ragged last wave): the split units' first segments read
+    h0 from a workspace copy at their own unit offsets."""
+    case = make_prefill(1, 512, 4, 64, 128, 1, 256, "bf16", h0_std=0.1, seed=16)
+    ssd.debug_force_prefill_split(2, 4)  # units 0, 1 whole; 2, 3 in four segments
+    try:
+        assert ssd.prefill_whole_units(1, 512, 4, 64, 128, 1, 256, ssd.SSD_BF16) == 2
+        y, hf, t = run_prefill(ssd, case)
+        h = t["h0"].clone()
+        y2, h2 = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=256, h0=h, h_final=h)
+        torch.cuda.synchronize()
+    finally:
+        ssd.debug_force_prefill_split(0, 0)
+    assert h2.data_ptr() == h.data_ptr()
+    assert torch.equal(y2, y) and torch.equal(h, hf)
+    y_ref, hf_ref = oracle_subset(case, [0], range(case.H))
+    check(_np(y2), y_ref, "bf16", "y")
+    check(_np(h), hf_ref, "bf16", "h_final")
+
+
 def test_back_to_back_chained_calls_match_single_calls():
     """Split prefills issued back to back on one stream and one workspace, alternating two
     inputs and in-place state updates, with no host synchronisation between them: the
