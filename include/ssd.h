@@ -87,7 +87,8 @@ SSD_API const char* ssd_last_error(void);
  *   h_t = exp(dt_t A) h_{t-1} + dt_t x_t B_t^T,  y_t = h_t C_t + D x_t,  h_{-1} = h0
  * through the chunked dual form.  T need not be a multiple of `chunk`: the last chunk
  * is then shorter.  T == 0 or b == 0 is a no-op apart from h_final = h0 (or zeros).
- * chunk must be 64, 128 or 256.  x, B, C, dt, A, D must not alias y or h_final.
+ * chunk must be 64, 128 or 256.  x, B, C, dt, A, D must not alias y or h_final, and the
+ * workspace (its required size from its start) must overlap no other buffer.
  * Arithmetic: SSD_BF16 inputs with P == 64 and N == 128 run one fused tensor-core kernel
  * (tcgen05 bf16 contractions, fp32 accumulation, fp32 decay in log space, fp32 running
  * state kept on chip), after a tensor-core state pass when (sequence, head) pairs would
@@ -105,7 +106,8 @@ SSD_API const char* ssd_last_error(void);
  * are the same (both depend on b * H and, on the fp32 path, on the chunk count).
  * The workspace's first 256 bytes hold a device status word (see ssd_prefill_check).
  * Errors: SSD_ERR_INVALID_ARG (null pointer for a required argument, negative size,
- * H % G != 0, bad chunk or dtype, misaligned pointer), SSD_ERR_UNSUPPORTED (P, N),
+ * H % G != 0, bad chunk or dtype, misaligned pointer, overlapping buffers other than
+ * h_final == h0), SSD_ERR_UNSUPPORTED (P, N),
  * SSD_ERR_WORKSPACE (workspace too small or NULL while required), SSD_ERR_CUDA.
  * ---------------------------------------------------------------------------------- */
 SSD_API size_t ssd_prefill_workspace_size(int b, int T, int H, int P, int N, int G, int chunk,
@@ -158,7 +160,8 @@ SSD_API size_t ssd_prefill_local_state_workspace_size(int b, int T, int H, int P
  * tensor-core state pass (the tokens cut into pieces to fill the SMs) and a fold of the
  * pieces.  T == 0 writes zeros.  Tensor-core shapes only: bf16, P = 64, N = 128.
  * Errors: SSD_ERR_INVALID_ARG (bad shape or pointer, outputs overlapping inputs or each
- * other), SSD_ERR_UNSUPPORTED (other dtypes or P, N), SSD_ERR_WORKSPACE, SSD_ERR_CUDA. */
+ * other, the workspace overlapping any of them), SSD_ERR_UNSUPPORTED (other dtypes or P,
+ * N), SSD_ERR_WORKSPACE, SSD_ERR_CUDA. */
 SSD_API int ssd_prefill_local_state(int b, int T, int H, int P, int N, int G, int io_dtype,
                                     const void* x, const float* dt, const float* A, const void* B,
                                     float* h_local, float* log_decay, void* workspace,

@@ -305,6 +305,8 @@ int ssd_prefill_local_state(int b, int T, int H, int P, int N, int G, int io_dty
     if (!aligned16(workspace)) return set_error(SSD_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
     for (const Range& o : outs)
         if (overlaps({workspace, need}, o)) return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps an output");
+    for (const Range& i : rin)
+        if (overlaps({workspace, need}, i)) return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps an input");
     return launch_prefill_tc_local_state(b, T, H, G, x, dt, A, B, h_local, log_decay, workspace, s);
 }
 
@@ -408,6 +410,8 @@ static int prefill_impl(int b, int T, int H, int P, int N, int G, int chunk, int
         return set_error(SSD_ERR_WORKSPACE, "workspace %zu bytes at %p, need %zu", workspace_bytes, workspace, need);
     if (!aligned16(workspace)) return set_error(SSD_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
     if (overlaps({workspace, need}, ry)) return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps y");
+    if (overlaps({workspace, need}, {h_final, h_final ? state_bytes : 0}))
+        return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps h_final");
     for (int i = 0; i < 7; ++i)
         if (overlaps({workspace, need}, rin[i])) return set_error(SSD_ERR_INVALID_ARG, "workspace overlaps %s", names[i]);
     if (use_tc(P, N, io_dtype))

@@ -89,6 +89,11 @@ def test_prefill_rejects_aliasing():
     h0 = ctypes.c_void_p(0x7000000000)
     hf = ctypes.c_void_p(0x7000000000 + 4096)  # partial overlap of h0 / h_final
     assert _prefill(ptrs=_fake(8), h0=h0, hf=hf) == INVALID
+    for io, N in [(0, 64), (1, 128)]:  # fp32 path, tensor-core path with a split workspace
+        p = _fake(8)
+        hf = ctypes.c_void_p(p[7].value + 256)  # h_final inside the workspace
+        assert _prefill(N=N, io=io, ptrs=p, hf=hf) == INVALID, io
+        assert "h_final" in ssd.last_error()
 
 
 def test_prefill_empty_batch_is_noop():
@@ -307,5 +312,7 @@ def test_context_parallel_entry_points_reject():
     assert L.ssd_prefill_local_state(1, 512, 4, 64, 128, 1, 0, x, dt, A, B, hl, ld, ws, 1 << 30, None) == UNSUP
     assert L.ssd_prefill_local_state(1, 512, 4, 64, 128, 1, 1, x, dt, A, B, None, ld, ws, 1 << 30, None) == INVALID
     assert L.ssd_prefill_local_state(1, 512, 4, 64, 128, 1, 1, x, dt, A, B, hl, ld, ws, 16, None) == WS
+    for inp in (x, dt, A, B):  # the workspace, written while the inputs are read, overlaps one
+        assert L.ssd_prefill_local_state(1, 512, 4, 64, 128, 1, 1, x, dt, A, B, hl, ld, inp, 1 << 30, None) == INVALID
     assert ssd.lib().ssd_prefill_local_state_workspace_size(1, 512, 4, 64, 128, 1, 1) > 0
     assert ssd.lib().ssd_prefill_local_state_workspace_size(1, 512, 4, 64, 64, 1, 1) == 0
