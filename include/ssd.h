@@ -266,8 +266,10 @@ SSD_API int ssd_prefill_whole_units(int b, int T, int H, int P, int N, int G, in
  * x, Bv, Cv = split(u); per head: h = exp(dt*A) h + dt * x Bv^T; y = h Cv + D x.
  * act is SSD_ACT_NONE or SSD_ACT_SILU; kconv must be 4.  The workspace (see
  * ssd_decode_workspace_size) holds per-(layer, sequence, group) arrival counters that
- * the call zero-fills itself; calls sharing one workspace must be stream-ordered.
- * Errors: as for ssd_prefill.
+ * the call zero-fills itself; calls sharing one workspace must be stream-ordered.  The
+ * buffers the step writes (h, conv_state, y, the workspace) must overlap neither one another
+ * nor any input; inputs may share memory with one another.
+ * Errors: as for ssd_prefill (SSD_ERR_INVALID_ARG for an overlap named above).
  * ---------------------------------------------------------------------------------- */
 SSD_API size_t ssd_decode_workspace_size(int layers, int b, int G);
 

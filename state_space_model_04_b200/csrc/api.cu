@@ -478,6 +478,33 @@ static int check_decode(int layers, int b, int H, int P, int N, int G, int kconv
     return SSD_OK;
 }
 
+// The buffers a decode step writes (h, conv_state, y and the workspace's arrival counters)
+// must not overlap one another or any buffer the step reads (xbc, dt, A, D, conv_w, conv_b);
+// for a plan, xbc, dt and y hold `ring` steps.
+static int check_decode_overlaps(int layers, int b, int H, int P, int N, int G, int kconv, int io_dtype,
+                                 const float* h, const float* conv_state, const void* xbc, const float* dt,
+                                 const float* A, const float* D, const float* conv_w, const float* conv_b,
+                                 const void* y, int ring, const void* ws) {
+    const size_t io_b = io_dtype == SSD_BF16 ? 2 : 4;
+    const size_t Dc = (size_t)H * P + 2 * (size_t)G * N, lb = (size_t)layers * b, R = (size_t)ring;
+    const Range writes[] = {{h, lb * H * P * N * 4}, {conv_state, lb * Dc * (kconv - 1) * 4},
+                            {y, R * lb * H * P * io_b}, {ws, decode_workspace_bytes(layers, b, G)}};
+    const Range reads[] = {{xbc, R * lb * Dc * io_b},         {dt, R * lb * H * 4},
+                           {A, (size_t)layers * H * 4},       {D, (size_t)layers * H * 4},
+                           {conv_w, (size_t)layers * Dc * kconv * 4}, {conv_b, (size_t)layers * Dc * 4}};
+    const char* wname[] = {"h", "conv_state", "y", "workspace"};
+    const char* rname[] = {"xbc", "dt", "A", "D", "conv_w", "conv_b"};
+    for (int i = 0; i < 4; ++i) {
+        for (int j = i + 1; j < 4; ++j)
+            if (overlaps(writes[i], writes[j]))
+                return set_error(SSD_ERR_INVALID_ARG, "%s overlaps %s", wname[i], wname[j]);
+        for (int j = 0; j < 6; ++j)
+            if (overlaps(writes[i], reads[j]))
+                return set_error(SSD_ERR_INVALID_ARG, "%s overlaps %s", wname[i], rname[j]);
+    }
+    return SSD_OK;
+}
+
 int ssd_decode_step(int layers, int b, int H, int P, int N, int G, int kconv, int act, int io_dtype,
                     float* h, float* conv_state, const void* xbc, const float* dt, const float* A,
                     const float* D, const float* conv_w, const float* conv_b, void* y,
@@ -489,17 +516,8 @@ int ssd_decode_step(int layers, int b, int H, int P, int N, int G, int kconv, in
     SSD_CHECK(check_ptr(xbc, "xbc", true));
     SSD_CHECK(check_ptr(dt, "dt", true));
     SSD_CHECK(check_ptr(y, "y", true));
-    const size_t io_b = io_dtype == SSD_BF16 ? 2 : 4;
-    const size_t Dc = (size_t)H * P + 2 * (size_t)G * N;
-    const Range ry{y, (size_t)layers * b * H * P * io_b};
-    const Range rh{h, (size_t)layers * b * H * P * N * 4};
-    const Range rc{conv_state, (size_t)layers * b * Dc * (kconv - 1) * 4};
-    const Range rin[] = {{xbc, (size_t)layers * b * Dc * io_b}, {dt, (size_t)layers * b * H * 4}};
-    if (overlaps(rh, rc) || overlaps(ry, rh) || overlaps(ry, rc))
-        return set_error(SSD_ERR_INVALID_ARG, "h, conv_state and y must not overlap");
-    for (const Range& r : rin)
-        if (overlaps(r, ry) || overlaps(r, rh) || overlaps(r, rc))
-            return set_error(SSD_ERR_INVALID_ARG, "an input overlaps h, conv_state or y");
+    SSD_CHECK(check_decode_overlaps(layers, b, H, P, N, G, kconv, io_dtype, h, conv_state, xbc, dt, A, D, conv_w,
+                                    conv_b, y, 1, workspace));
     return launch_decode_step(layers, b, H, N, G, act, io_dtype, h, conv_state, xbc, dt, A, D, conv_w,
                               conv_b, y, workspace, static_cast<cudaStream_t>(stream));
 }
@@ -538,6 +556,8 @@ int ssd_decode_plan_create(ssd_decode_plan** plan, int layers, int b, int H, int
     SSD_CHECK(check_ptr(xbc_ring, "xbc_ring", true));
     SSD_CHECK(check_ptr(dt_ring, "dt_ring", true));
     SSD_CHECK(check_ptr(y_ring, "y_ring", true));
+    SSD_CHECK(check_decode_overlaps(layers, b, H, P, N, G, kconv, io_dtype, h, conv_state, xbc_ring, dt_ring, A, D,
+                                    conv_w, conv_b, y_ring, ring, workspace));
     return create_decode_plan(plan, layers, b, H, N, G, act, io_dtype, h, conv_state, xbc_ring, dt_ring,
                               ring, A, D, conv_w, conv_b, y_ring, n_steps, workspace);
 }

@@ -134,6 +134,12 @@ def test_decode_null_aliasing_and_empty():
     p = _fake(10)
     p[8] = p[0]  # y aliases h
     assert _decode(ptrs=p) == INVALID
+    # a written buffer (h 0, conv_state 1, y 8, workspace 9) overlapping anything else
+    for w, other in [(9, 0), (9, 1), (9, 2), (9, 4), (0, 4), (1, 6), (8, 7), (8, 3)]:
+        p = _fake(10)
+        p[w] = ctypes.c_void_p(p[other].value + 16)  # inside even the 32-byte A, D and dt
+        assert _decode(ptrs=p) == INVALID, (w, other)
+        assert "overlaps" in ssd.last_error()
     assert _decode(b=0) == OK
     assert _decode(layers=0) == OK
 
@@ -151,6 +157,15 @@ def test_decode_plan_rejects():
     assert st == INVALID
     assert L.ssd_decode_plan_create(None, 1, 1, 4, 64, 128, 1, 4, 1, 1, f[0], f[1], f[2], f[3], 2,
                                     f[4], f[5], f[6], f[7], f[8], 8, f[9], 1 << 20) == INVALID
+    # a written buffer overlapping a ring or the weights: y_ring inside xbc_ring's second
+    # step, the workspace inside conv_w
+    g = _fake(10)
+    y_in_ring = ctypes.c_void_p(g[2].value + 1 * 4 * 64 * 2 + 2 * 128 * 2 * 2)
+    assert L.ssd_decode_plan_create(ctypes.byref(handle), 1, 1, 4, 64, 128, 1, 4, 1, 1, g[0], g[1], g[2], g[3], 2,
+                                    g[4], g[5], g[6], g[7], y_in_ring, 8, g[9], 1 << 20) == INVALID
+    assert L.ssd_decode_plan_create(ctypes.byref(handle), 1, 1, 4, 64, 128, 1, 4, 1, 1, g[0], g[1], g[2], g[3], 2,
+                                    g[4], g[5], g[6], g[7], g[8], 8, g[6], 1 << 20) == INVALID
+    assert not handle.value
     assert L.ssd_decode_plan_launch(None, None) == INVALID
     assert L.ssd_decode_plan_destroy(None) == OK
     # the one-call loop runs the same checks before anything is built or enqueued
