@@ -126,6 +126,18 @@ def profile_end(max_entries=64):
     return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms) for i in range(n)}
 
 
+def _check_device(device, **tensors):
+    """Every tensor of one call must sit on the GPU of its first operand, and that GPU must be
+    the current device: the library launches there and its kernels read these pointers
+    directly (a tensor on another GPU would be a peer address)."""
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError("%s is on %s, the call's other tensors on %s" % (name, t.device, device))
+    if device.type == "cuda" and device.index is not None and device.index != torch.cuda.current_device():
+        raise ValueError("the tensors are on %s but the current device is cuda:%d (call under "
+                         "torch.cuda.device(...))" % (device, torch.cuda.current_device()))
+
+
 def _check(status: int, where: str):
     if status != SSD_OK:
         raise SSDError(status, where, last_error())
@@ -198,6 +210,8 @@ def prefill(x, dt, A, B, C, D, chunk=256, h0=None, y=None, h_final=None, workspa
     need = prefill_workspace_size(b, T, H, P, N, G, chunk, io)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check_device(x.device, dt=dt, A=A, B=B, C=C, D=D, h0=h0, y=y, h_final=h_final, dt_bias=dt_bias,
+                  workspace=workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     if dt_raw:
         st = lib().ssd_prefill_dt_raw(b, T, H, P, N, G, int(chunk), io, _ptr(x), _ptr(dt), _ptr(dt_bias),
@@ -247,6 +261,7 @@ def prefill_local_state(x, dt, A, B, h_local=None, log_decay=None, workspace=Non
     need = int(lib().ssd_prefill_local_state_workspace_size(b, T, H, P, N, G, SSD_BF16))
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check_device(x.device, dt=dt, A=A, B=B, h_local=h_local, log_decay=log_decay, workspace=workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().ssd_prefill_local_state(b, T, H, P, N, G, SSD_BF16, _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
                                        _ptr(h_local), _ptr(log_decay), _ptr(workspace), ws_bytes, _stream(stream))
@@ -265,6 +280,7 @@ def prefill_context_scan(rank, h_local_all, log_decay_all, h0=None, h_in=None, s
     if h_in is None:
         h_in = torch.empty((b, H, P, N), dtype=torch.float32, device=h_local_all.device)
     _need(h_in, "h_in", torch.float32, (b, H, P, N))
+    _check_device(h_local_all.device, log_decay_all=log_decay_all, h0=h0, h_in=h_in)
     st = lib().ssd_prefill_context_scan(world, int(rank), b, H, P, N, _ptr(h0), _ptr(h_local_all),
                                         _ptr(log_decay_all), _ptr(h_in), _stream(stream))
     _check(st, "ssd_prefill_context_scan")
@@ -335,6 +351,8 @@ def decode_step(h, conv_state, xbc, dt, A, D, conv_w, conv_b, G=1, act=SSD_ACT_S
     _need(y, "y", xbc.dtype, (layers, b, H, P))
     if workspace is None:
         workspace = torch.empty(decode_workspace_size(layers, b, G), dtype=torch.uint8, device=h.device)
+    _check_device(h.device, conv_state=conv_state, xbc=xbc, dt=dt, A=A, D=D, conv_w=conv_w, conv_b=conv_b, y=y,
+                  workspace=workspace)
     st = lib().ssd_decode_step(layers, b, H, P, N, G, k, act, io, _ptr(h), _ptr(conv_state), _ptr(xbc),
                                _ptr(dt), _ptr(A), _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(y),
                                _ptr(workspace), workspace.numel(), _stream(stream))
@@ -352,6 +370,7 @@ def decode_step_noalloc(h, conv_state, xbc, dt, A, D, conv_w, conv_b, y, G=1, ac
     io = _io(xbc)
     _need(dt, "dt", torch.float32, (layers, b, H))
     _need(y, "y", xbc.dtype, (layers, b, H, P))
+    _check_device(h.device, conv_state=conv_state, xbc=xbc, dt=dt, A=A, D=D, conv_w=conv_w, conv_b=conv_b, y=y)
     st = lib().ssd_decode_step_noalloc(layers, b, H, P, N, G, k, act, io, _ptr(h), _ptr(conv_state),
                                        _ptr(xbc), _ptr(dt), _ptr(A), _ptr(D), _ptr(conv_w), _ptr(conv_b),
                                        _ptr(y), _stream(stream))
@@ -374,6 +393,8 @@ class DecodePlan:
         if y_ring is None:
             y_ring = torch.empty((ring, layers, b, H, P), dtype=xbc_ring.dtype, device=h.device)
         _need(y_ring, "y_ring", xbc_ring.dtype, (ring, layers, b, H, P))
+        _check_device(h.device, conv_state=conv_state, xbc_ring=xbc_ring, dt_ring=dt_ring, A=A, D=D,
+                      conv_w=conv_w, conv_b=conv_b, y_ring=y_ring)
         self.workspace = torch.empty(decode_workspace_size(layers, b, G), dtype=torch.uint8, device=h.device)
         self._keep = (h, conv_state, xbc_ring, dt_ring, A, D, conv_w, conv_b, y_ring)
         self.y_ring = y_ring
@@ -414,6 +435,8 @@ def decode_loop(h, conv_state, xbc_ring, dt_ring, A, D, conv_w, conv_b, n_steps,
     _need(xbc_ring, "xbc_ring", None, (ring, layers, b, Dc))
     io = _io(xbc_ring)
     _need(dt_ring, "dt_ring", torch.float32, (ring, layers, b, H))
+    _check_device(h.device, conv_state=conv_state, xbc_ring=xbc_ring, dt_ring=dt_ring, A=A, D=D,
+                  conv_w=conv_w, conv_b=conv_b)
     y_ring = torch.empty((ring, layers, b, H, P), dtype=xbc_ring.dtype, device=h.device)
     ws = torch.empty(decode_workspace_size(layers, b, G), dtype=torch.uint8, device=h.device)
     st = lib().ssd_decode_loop(layers, b, H, P, N, G, k, act, io, _ptr(h), _ptr(conv_state), _ptr(xbc_ring),

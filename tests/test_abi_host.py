@@ -185,6 +185,18 @@ def test_binding_refuses_cpu_tensors():
                     torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16), torch.zeros(4))
 
 
+def test_binding_refuses_tensors_on_another_device():
+    """Every tensor of a call must sit on the device of its first operand (the kernels read
+    the pointers directly; a tensor on another GPU would be a peer address).  The check runs
+    before the library is called; None operands are skipped."""
+    import torch
+    from state_space_model_04_b200.ssd import _check_device
+    a = torch.zeros(4)
+    _check_device(a.device, b=torch.zeros(2), c=None)
+    with pytest.raises(ValueError, match="c is on meta"):
+        _check_device(a.device, b=torch.zeros(2), c=torch.empty(2, device="meta"))
+
+
 def test_segment_hook_and_workspace():
     """The split of a sequence into segments sizes the workspace: one fp32 state and one
     log decay per (sequence, head) for every segment but the last."""
