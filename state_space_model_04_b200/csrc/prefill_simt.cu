@@ -563,14 +563,16 @@ chunk_output_small_kernel(int T, int H, int G, int L, int nc, int ks, const IoT*
     }
 }
 
+// SMs of the device current at the first call (148 when no device answers); initialised
+// once, thread-safely
 int sm_count_simt() {
-    static int n = 0;
-    if (n <= 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            n <= 0)
-            n = 148;
-    }
+    static const int n = [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            v <= 0)
+            v = 148;
+        return v;
+    }();
     return n;
 }
 

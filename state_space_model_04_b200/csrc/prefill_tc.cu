@@ -1412,14 +1412,16 @@ namespace {
 constexpr size_t kSegOffset = 512;  // status word and launch scratch come first
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// SMs of the device current at the first call (148 when no device answers); initialised
+// once, thread-safely
 int sm_count() {
-    static int n = 0;
-    if (n <= 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            n <= 0)
-            n = 148;
-    }
+    static const int n = [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            v <= 0)
+            v = 148;
+        return v;
+    }();
     return n;
 }
 
